@@ -1,0 +1,379 @@
+"""Benchmark of the exact tiled attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload dense_causal|packed_causal|long_outlier|mxfp8_packed]
+
+One step = one ``attn_fwd`` call through the C ABI (the schedule-build
+kernel, the MXFP8 pre-pass for the MXFP8 workload, and the attention
+kernel) over the workload's whole batch, inputs resident in HBM.  Prints one
+JSON line (rank 0).  Throughput is TFLOP/s with the causal FLOP convention
+4 L^2 d / 2 per head and document.  Under torchrun each rank runs the same
+workload on its own GPU (independent replicas, weak scaling: the path has no
+cross-GPU exchange); the time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload and prints the same metric (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_tiled_attention_39_b200 import workloads  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (causal, bf16 & MXFP8) and % of B200 dense tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [x for x in sm if x >= 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def bench_ours(args):
+    from exact_tiled_attention_39_b200 import attn as A
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    w = workloads.get(args.workload)
+    inp = workloads.make_inputs(w)
+    T, H, d = inp["q"].shape
+    causal = True
+    dtype = A.ATTN_MXFP8 if w.dtype == "mxfp8" else A.ATTN_BF16
+    lengths = inp["lengths"]
+    max_seqlen = max(lengths)
+    flops = workloads.flops(lengths, H, d, causal)
+
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    cu = inp["cu_seqlens"].to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+    ws = A.make_workspace(A.Shape(T, len(lengths), H, d, max_seqlen), dtype, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        A.attn_fwd(q, k, v, cu, out, lse, causal, inp["scale"], dtype=dtype, stream=stream,
+                   workspace=ws, max_seqlen=max_seqlen)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert A.attn_get_device_error(ws) == 0, "device error during warm-up"
+
+    # ---- device-timed region: K steps, barrier + sync on both sides
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    ms_total = t0.elapsed_time(t1)
+    if pg:
+        tt = torch.tensor([ms_total], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    err = A.attn_get_device_error(ws)
+    value = world * flops / (ms_step * 1e-3) / 1e12
+
+    # ---- per-launch timing of the step on its own stream (roofline)
+    per = []
+    for _ in range(5):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        per.append(e0.elapsed_time(e1))
+    per_ms = statistics.median(per)
+
+    # ---- end to end through the public API: pinned host in, host out
+    hq, hk, hv = (inp[n].pin_memory() for n in ("q", "k", "v"))
+    hcu = inp["cu_seqlens"].pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        cu.copy_(hcu, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = s0.elapsed_time(s1) / e2e_steps
+    if pg:
+        tt = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcu))
+    d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    timed_s = ms_total * 1e-3
+    peak_key = "bf16_tflops_sustained" if timed_s > 1.0 else "bf16_tflops"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    if dtype == A.ATTN_MXFP8:
+        peak *= 2.0        # fp8 dense peak = 2 x bf16 (nominal ratio)
+    achieved = flops / (per_ms * 1e-3) / 1e12
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "mxfp8" if dtype == A.ATTN_MXFP8 else "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, see workloads.py)",
+        "config": {
+            "workload": f"{w.name}: {w.description}",
+            "tokens": T, "heads": H, "head_dim": d, "docs": len(lengths),
+            "causal": causal, "flops_per_step": flops,
+            "l2": f"inputs {3 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2; no flush",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "peak_source": f"{peak_source_name(peak_key, dtype)} ({peak_src})",
+            "timed_unit": "one attn_fwd call (schedule kernel + attention kernel), median of 5",
+            "traffic": None,
+        },
+        "e2e": {
+            "value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s",
+            "ms_per_step": round(e2e_ms, 3),
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+        },
+        "gpu_launches": args.steps * (3 if dtype == A.ATTN_MXFP8 else 2),
+        "clocks": clk.summary(),
+        "device_error": err,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_budget)
+    return line
+
+
+def peak_source_name(key, dtype):
+    base = {"bf16_tflops": "bf16 burst", "bf16_tflops_sustained": "bf16 sustained"}[key]
+    return base + (" x2 for fp8" if dtype == 1 else "")
+
+
+def cpu_baseline(w, inp, budget_s=15.0):
+    """Time the fp64 oracle on the host cores on a bounded sample of the
+    workload: whole (document, head) problems, as many as fit the budget."""
+    from oracle.attention import ref_attention
+    from oracle.mxfp8 import quantize_mxfp8_ref, dequantize_mxfp8_ref
+
+    cores = len(os.sched_getaffinity(0))
+    torch.set_num_threads(cores)
+    lengths = inp["lengths"]
+    starts = np.concatenate([[0], np.cumsum(lengths)])
+    H, d = inp["q"].shape[1], inp["q"].shape[2]
+    # order: documents first, heads second, largest documents first
+    problems = [(i, h) for i in np.argsort(lengths)[::-1] for h in range(H)]
+    done_flops, done = 0.0, 0
+    t_start = time.perf_counter()
+    for i, h in problems:
+        a, b = int(starts[i]), int(starts[i + 1])
+        q = inp["q"][a:b, h:h + 1].double().numpy()
+        k = inp["k"][a:b, h:h + 1].double().numpy()
+        v = inp["v"][a:b, h:h + 1].double().numpy()
+        if w.dtype == "mxfp8":
+            q, k, v = (dequantize_mxfp8_ref(*quantize_mxfp8_ref(x)) for x in (q, k, v))
+        ref_attention(q, k, v, [0, b - a], True, inp["scale"])
+        done_flops += workloads.flops([b - a], 1, d, True)
+        done += 1
+        if time.perf_counter() - t_start > budget_s:
+            break
+    el = time.perf_counter() - t_start
+    return {"value": round(done_flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{done} of {len(problems)} (document, head) problems, fp64, "
+                      f"{el:.1f} s"}
+
+
+def bench_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    w = workloads.get(args.workload)
+    inp = workloads.make_inputs(w)
+    budget = max(2.0, args.cpu_budget / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(w, inp, budget_s=budget)
+    vals = [cpu_baseline(w, inp, budget_s=budget) for _ in range(args.steps)]
+    v = statistics.median(x["value"] for x in vals)
+    T, H, d = inp["q"].shape
+    flops = workloads.flops(inp["lengths"], H, d, True)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": v,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(flops / (v * 1e12) * 1e3, 3) if v else None,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16, see workloads.py)",
+        "config": {"workload": f"{w.name}: {w.description}", "tokens": T, "heads": H,
+                   "head_dim": d, "causal": True, "flops_per_step": flops},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": vals[0]["cores"],
+                         "kind": "oracle", "sample": vals[0]["sample"] + " per step"},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="dense_causal", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        line = bench_reference(args)
+    else:
+        from exact_tiled_attention_39_b200 import build
+        if dist_env()[1] == 0 or not os.path.exists(build.LIB):
+            build.build()
+        line = bench_ours(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

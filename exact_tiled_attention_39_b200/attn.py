@@ -1,0 +1,168 @@
+"""Thin ctypes binding over ``libattn.so`` (C ABI in ``include/attn.h``).
+
+Argument marshalling only: torch tensors provide device memory and streams;
+every step of the computation runs in the library's CUDA kernels.  There is
+no CPU path: if the library is missing or a GPU is absent, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = ["ATTN_BF16", "ATTN_MXFP8", "AttnError", "lib", "workspace_size", "attn_fwd",
+           "attn_quantize_mxfp8", "attn_get_device_error", "status_string", "make_workspace",
+           "LIB_PATH", "EXPORTED_SYMBOLS"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
+
+ATTN_BF16 = 0
+ATTN_MXFP8 = 1
+
+STATUS = {
+    0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_ALIGNMENT",
+    4: "ATTN_ERR_WORKSPACE", 5: "ATTN_ERR_BAD_SEQLENS", 6: "ATTN_ERR_TIMEOUT", 7: "ATTN_ERR_CUDA",
+}
+
+EXPORTED_SYMBOLS = ("attn_workspace_size", "attn_fwd", "attn_quantize_mxfp8",
+                    "attn_get_device_error", "attn_status_string", "attn_abi_version")
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("total_tokens", ctypes.c_int32), ("num_seqs", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("max_seqlen", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m exact_tiled_attention_39_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        L.attn_workspace_size.argtypes = [ctypes.POINTER(_Shape), ctypes.c_int]
+        L.attn_workspace_size.restype = sz
+        L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                               vp, ctypes.POINTER(_Shape), vp, sz]
+        L.attn_fwd.restype = ctypes.c_int
+        L.attn_quantize_mxfp8.argtypes = [vp, vp, vp, i64, i32, vp]
+        L.attn_quantize_mxfp8.restype = ctypes.c_int
+        L.attn_get_device_error.argtypes = [vp, vp, ctypes.POINTER(i32)]
+        L.attn_get_device_error.restype = ctypes.c_int
+        L.attn_status_string.argtypes = [ctypes.c_int]
+        L.attn_status_string.restype = ctypes.c_char_p
+        L.attn_abi_version.argtypes = []
+        L.attn_abi_version.restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().attn_status_string(code).decode()
+
+
+@dataclass(frozen=True)
+class Shape:
+    total_tokens: int
+    num_seqs: int
+    num_heads: int
+    head_dim: int
+    max_seqlen: int
+
+    def c(self) -> _Shape:
+        return _Shape(self.total_tokens, self.num_seqs, self.num_heads, self.head_dim,
+                      self.max_seqlen)
+
+
+def workspace_size(shape: Shape, dtype: int = ATTN_BF16) -> int:
+    s = shape.c()
+    return int(lib().attn_workspace_size(ctypes.byref(s), dtype))
+
+
+def make_workspace(shape: Shape, dtype: int = ATTN_BF16, device=None) -> torch.Tensor:
+    n = workspace_size(shape, dtype)
+    if n == 0:
+        raise AttnError(1, "attn_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def attn_fwd(q, k, v, cu_seqlens, out, lse, causal: bool, scale: float, dtype: int = ATTN_BF16,
+             stream=None, workspace=None, max_seqlen: int | None = None,
+             num_seqs: int | None = None):
+    """Run the forward through the C ABI.  q, k, v, out: bf16 [T, H, d]
+    (contiguous, CUDA); lse: fp32 [H, T]; cu_seqlens: int32 CUDA tensor or
+    None (dense: ``num_seqs`` documents of ``max_seqlen`` tokens).  With
+    cu_seqlens, ``max_seqlen`` must bound every document length (a longer
+    one is reported by the device as ATTN_ERR_BAD_SEQLENS).  Returns the
+    workspace used (allocated if not given)."""
+    T, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (H, T):
+        raise ValueError("lse must be a contiguous fp32 tensor of shape [H, T]")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+            raise ValueError("cu_seqlens must be an int32 CUDA tensor")
+        ns = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens (no host sync is done)")
+    else:
+        ns = num_seqs if num_seqs is not None else 1
+        if max_seqlen is None:
+            max_seqlen = T // max(ns, 1)
+    shape = Shape(T, ns, H, d, int(max_seqlen))
+    if workspace is None:
+        workspace = make_workspace(shape, dtype, q.device)
+    s = shape.c()
+    rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(out), _ptr(lse),
+                        int(bool(causal)), float(scale), int(dtype),
+                        _stream_handle(stream, q.device), ctypes.byref(s), _ptr(workspace),
+                        workspace.numel())
+    if rc != 0:
+        raise AttnError(rc, "attn_fwd")
+    return workspace
+
+
+def attn_quantize_mxfp8(x, codes, scales, stream=None):
+    """E4M3 + E8M0 quantisation of a bf16 [rows, cols] CUDA tensor (any
+    leading shape; the last dimension is ``cols``)."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    rc = lib().attn_quantize_mxfp8(_ptr(x), _ptr(codes), _ptr(scales), rows, cols,
+                                   _stream_handle(stream, x.device))
+    if rc != 0:
+        raise AttnError(rc, "attn_quantize_mxfp8")
+
+
+def attn_get_device_error(workspace, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    rc = lib().attn_get_device_error(_ptr(workspace), _stream_handle(stream, workspace.device),
+                                     ctypes.byref(v))
+    if rc != 0:
+        raise AttnError(rc, "attn_get_device_error")
+    return int(v.value)

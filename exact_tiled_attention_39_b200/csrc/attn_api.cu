@@ -1,0 +1,247 @@
+// Host side of the C ABI declared in include/attn.h: argument checks,
+// workspace carving, TMA tensor-map encoding and the kernel launches.
+// Everything is asynchronous on the caller's stream; nothing is allocated.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn_fwd_bf16.cuh"
+#include "common.cuh"
+#include "quant_mxfp8.cuh"
+#include "schedule.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kScheduleThreads = 1024;
+constexpr int kSortCapacityMax = 16384;                   // 128 KB of keys
+constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;  // 1 s per wait
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t sort_capacity_for(int64_t max_entries) {
+  int64_t c = 1;
+  while (c < max_entries) c <<= 1;
+  return c > kSortCapacityMax ? 0 : c;
+}
+
+struct WsLayout {
+  size_t sorted_off, unsorted_off, mx_off, total;
+  int64_t max_entries;
+};
+
+WsLayout ws_layout(const attn_shape_t& s, attn_dtype_t dtype) {
+  WsLayout w{};
+  w.max_entries = max_work_entries(s.total_tokens, s.num_seqs);
+  w.sorted_off = kWsListOffset;
+  w.unsorted_off = align_up(w.sorted_off + 16 * static_cast<size_t>(w.max_entries), kWsAlign);
+  w.mx_off = align_up(w.unsorted_off + 16 * static_cast<size_t>(w.max_entries), kWsAlign);
+  w.total = w.mx_off;
+  if (dtype == ATTN_MXFP8) {
+    const size_t elems = static_cast<size_t>(s.total_tokens) * s.num_heads * s.head_dim;
+    w.total += 3 * align_up(elems, kWsAlign) + 3 * align_up(elems / 32, kWsAlign);
+  }
+  return w;
+}
+
+attn_status_t check_shape(const attn_shape_t* s) {
+  if (s == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (s->total_tokens < 0 || s->num_seqs < 0 || s->num_heads < 1 || s->max_seqlen < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (s->head_dim != 64 && s->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
+  if (s->total_tokens > 0 && s->num_seqs < 1) return ATTN_ERR_INVALID_ARG;
+  const int64_t elems = static_cast<int64_t>(s->total_tokens) * s->num_heads;
+  if (elems > (int64_t(1) << 31)) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+attn_status_t device_info(int* dev_out, DeviceInfo* info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return ATTN_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (cudaFuncSetAttribute(attn_fwd_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FwdLayout<64>::kAllocBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_bf16_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FwdLayout<128>::kAllocBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(build_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSortCapacityMax * 8) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    d.ready = true;
+  }
+  *dev_out = dev;
+  *info = d;
+  return ATTN_OK;
+}
+
+// 3-D map over a [T, H, d] bf16 tensor: box = 64 head-dim elements (128 B,
+// the swizzle span) x 1 head x 128 tokens, 128-byte swizzle, zero fill.
+bool encode_qkv_map(CUtensorMap* m, const void* base, int T, int H, int d) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(H) * d * 2};
+  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kBlockM)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+int32_t attn_abi_version(void) { return ATTN_ABI_VERSION; }
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_ALIGNMENT: return "ATTN_ERR_ALIGNMENT";
+    case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+    case ATTN_ERR_BAD_SEQLENS: return "ATTN_ERR_BAD_SEQLENS";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+  }
+  return "ATTN_ERR_UNKNOWN";
+}
+
+size_t attn_workspace_size(const attn_shape_t* shape, attn_dtype_t dtype) {
+  if (check_shape(shape) != ATTN_OK) return 0;
+  if (dtype != ATTN_BF16 && dtype != ATTN_MXFP8) return 0;
+  return ws_layout(*shape, dtype).total;
+}
+
+attn_status_t attn_quantize_mxfp8(const void* x, uint8_t* codes, uint8_t* scales, int64_t rows,
+                                  int32_t cols, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 32 != 0) return ATTN_ERR_INVALID_ARG;
+  if (rows == 0) return ATTN_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes)) return ATTN_ERR_ALIGNMENT;
+  const long long n_blocks = rows * static_cast<long long>(cols / 32);
+  const int threads = 256;
+  const long long grid = (n_blocks + threads - 1) / threads;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  quantize_mxfp8_kernel<<<static_cast<unsigned>(grid), threads, 0,
+                          static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(x), reinterpret_cast<uint4*>(codes), scales, n_blocks);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                       void* out, float* lse, int causal, float scale, attn_dtype_t dtype,
+                       void* stream, const attn_shape_t* shape, void* workspace,
+                       size_t workspace_bytes) {
+  const attn_status_t st = check_shape(shape);
+  if (st != ATTN_OK) return st;
+  if (dtype != ATTN_BF16 && dtype != ATTN_MXFP8) return ATTN_ERR_UNSUPPORTED;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  const attn_shape_t s = *shape;
+  if (cu_seqlens == nullptr &&
+      static_cast<int64_t>(s.num_seqs) * s.max_seqlen != static_cast<int64_t>(s.total_tokens))
+    return ATTN_ERR_INVALID_ARG;
+  if (s.total_tokens == 0) return ATTN_OK;
+  if (!q || !k || !v || !out || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return ATTN_ERR_ALIGNMENT;
+  const WsLayout wl = ws_layout(s, dtype);
+  if (workspace == nullptr || workspace_bytes < wl.total) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+  if (dtype == ATTN_MXFP8) return ATTN_ERR_UNSUPPORTED;
+
+  int dev = 0;
+  DeviceInfo info;
+  if (device_info(&dev, &info) != ATTN_OK) return ATTN_ERR_CUDA;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* header = reinterpret_cast<int32_t*>(ws);
+
+  // 1. schedule (validates cu_seqlens, writes the work list and its length)
+  const int64_t cap = sort_capacity_for(wl.max_entries);
+  build_schedule_kernel<<<1, kScheduleThreads, static_cast<size_t>(cap) * 8, strm>>>(
+      cu_seqlens, s.num_seqs, s.total_tokens, s.max_seqlen, s.max_seqlen, causal, header,
+      reinterpret_cast<int4*>(ws + wl.sorted_off), reinterpret_cast<int4*>(ws + wl.unsorted_off),
+      static_cast<int>(cap));
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+  // 2. attention
+  CUtensorMap tq, tk, tv;
+  if (!encode_qkv_map(&tq, q, s.total_tokens, s.num_heads, s.head_dim) ||
+      !encode_qkv_map(&tk, k, s.total_tokens, s.num_heads, s.head_dim) ||
+      !encode_qkv_map(&tv, v, s.total_tokens, s.num_heads, s.head_dim))
+    return ATTN_ERR_CUDA;
+  FwdParams fp;
+  fp.out = out;
+  fp.lse = lse;
+  fp.ws_header = header;
+  fp.work = reinterpret_cast<const int4*>(ws + wl.sorted_off);
+  fp.err = header + kWsErrorOffset / 4;
+  fp.total_tokens = s.total_tokens;
+  fp.num_heads = s.num_heads;
+  fp.causal = causal;
+  fp.scale_log2 = scale * 1.4426950408889634f;
+  fp.timeout_ns = kWaitTimeoutNs;
+  const int64_t max_units = wl.max_entries * s.num_heads;
+  const int grid = static_cast<int>(max_units < info.num_sms ? max_units : info.num_sms);
+  if (s.head_dim == 128) {
+    attn_fwd_bf16_kernel<128><<<grid, 384, FwdLayout<128>::kAllocBytes, strm>>>(tq, tk, tv, fp);
+  } else {
+    attn_fwd_bf16_kernel<64><<<grid, 384, FwdLayout<64>::kAllocBytes, strm>>>(tq, tk, tv, fp);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_get_device_error(const void* workspace, void* stream, int32_t* device_status) {
+  if (workspace == nullptr || device_status == nullptr) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(strm) != cudaSuccess) return ATTN_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const int32_t zero = 0;
+  if (cudaMemcpy(const_cast<void*>(workspace), &zero, sizeof(zero), cudaMemcpyHostToDevice) !=
+      cudaSuccess)
+    return ATTN_ERR_CUDA;
+  *device_status = v;
+  return ATTN_OK;
+}
+
+}  // extern "C"

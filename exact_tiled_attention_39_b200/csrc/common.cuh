@@ -1,0 +1,34 @@
+// Constants shared by the host launcher and the device kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/attn.h"
+
+namespace attn {
+
+constexpr int kBlockM = 128;        // query rows per tile (one TMEM lane per row)
+constexpr int kBlockN = 128;        // keys per key/value tile
+constexpr int kTilesPerUnit = 2;    // query tiles per work unit (ping-pong pair)
+constexpr int kRowsPerUnit = kBlockM * kTilesPerUnit;
+
+// Workspace layout: a 256-byte header, then the work list.
+constexpr size_t kWsErrorOffset = 0;     // int32 error word (attn_status_t)
+constexpr size_t kWsCountOffset = 4;     // int32 number of work-list entries
+constexpr size_t kWsListOffset = 256;    // int4 entries
+constexpr size_t kWsAlign = 256;
+
+// Lazy rescaling threshold in log2 units: the output accumulator keeps a
+// stale maximum until the row maximum has grown by more than this, so the
+// unnormalised weights stay below 2^kRescaleTau.
+constexpr float kRescaleTau = 8.0f;
+
+// Upper bound of the work-list length: every document contributes
+// ceil(L / 256) <= L / 256 + 1 entries.
+inline int64_t max_work_entries(int64_t total_tokens, int64_t num_seqs) {
+  return total_tokens / kRowsPerUnit + num_seqs + 1;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace attn

@@ -1,0 +1,139 @@
+/*
+ * attn.h - C ABI of the exact tiled attention forward for NVIDIA B200
+ * (sm_100a).  Library: exact_tiled_attention_39_b200/libattn.so.
+ *
+ * What is computed
+ * ----------------
+ * For every document D of a packed batch and every head h:
+ *     S = scale * Q_D K_D^T            (rows: queries, columns: keys of D)
+ *     S_ij = -inf  unless  (!causal || j <= i)    (indices relative to D)
+ *     P = row-softmax(S),  O = P V_D,  lse_i = max_j S_ij + ln sum_j exp(S_ij - max_j S_ij)
+ * "FlashAttention và IO" (aihero.vn), section "Ma trận trung gian là một
+ * khoản chi phí", defines the dense computation (score matrix, softmax,
+ * product with V).  Section "Tiling giữ công việc ở gần nơi tính" requires
+ * that neither S nor P is ever written to device memory, and section
+ * "Softmax qua nhiều khối cần thống kê chạy" gives the running statistics
+ * (maximum m, normaliser l, weighted sum u, old part multiplied by
+ * exp(m - m_new), result u / l) by which the kernel gets the exact result
+ * tile by tile.  "FlashAttention, pelatihan multi-GPU, dan kuantisasi bobot"
+ * (indonesian.itimpress.au), section 1, gives the loop order (outer loop
+ * over query blocks, inner over key/value blocks), asynchronous tile copies
+ * and producer / consumer warp roles.  The MXFP8 variant follows "FLAMIA:
+ * Blackwell Üzerinde Hızlı ve Nedensel Olarak Güvenli Eğitim İçin Flash
+ * Mikro-Ölçeklemeli Dikkat Mekanizması" (blog.edumints.com), section
+ * "FLAMIA Mimarisi ve Temel Tasarım İlkeleri": fused quantisation, packed
+ * documents used in place, and scales that never let a future token
+ * influence the past (here: one scale per token, head and 32 head-dim
+ * elements).
+ *
+ * Layouts (all row-major, contiguous)
+ * -----------------------------------
+ *   q, k, v, out : bf16 [T, H, d]  (token, head, head-dim); token stride H*d.
+ *   lse          : fp32 [H, T].
+ *   cu_seqlens   : int32 [num_seqs + 1] in DEVICE memory: 0 = cu[0] <=
+ *                  cu[1] <= ... <= cu[num_seqs] = T; document i is tokens
+ *                  [cu[i], cu[i+1]).  NULL means dense: num_seqs documents
+ *                  of max_seqlen tokens each, T = num_seqs * max_seqlen.
+ *
+ * Conventions
+ * -----------
+ *   - All tensor pointers are device pointers owned by the caller and must be
+ *     16-byte aligned; they must stay valid until the stream work completes.
+ *     The library allocates nothing and keeps no state between calls except
+ *     a per-device cache of kernel attributes.
+ *   - Supported: d in {64, 128}; H >= 1; T < 2^31; scale finite and > 0.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Host-checkable faults return a non-OK status
+ *     before anything is launched.  Faults in the contents of cu_seqlens are
+ *     found on the device: the call then records ATTN_ERR_BAD_SEQLENS in the
+ *     workspace's error word and leaves out and lse untouched.  Every wait
+ *     inside the kernels is bounded; if one runs out the kernel records
+ *     ATTN_ERR_TIMEOUT and returns.  attn_get_device_error reads the word.
+ *   - T == 0 is a no-op that returns ATTN_OK.  Empty documents are allowed.
+ */
+#ifndef EXACT_TILED_ATTENTION_ATTN_H
+#define EXACT_TILED_ATTENTION_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ATTN_ABI_VERSION 1
+
+typedef enum {
+  ATTN_BF16 = 0,  /* bf16 operands, bf16 tensor-core products, fp32 softmax   */
+  ATTN_MXFP8 = 1  /* bf16 inputs quantised in-call to E4M3 + E8M0 (per token,
+                     head and 32 head-dim elements), block-scaled products    */
+} attn_dtype_t;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,  /* NULL pointer, negative size, bad scale, ...   */
+  ATTN_ERR_UNSUPPORTED = 2,  /* head_dim or dtype not supported               */
+  ATTN_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned              */
+  ATTN_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than required       */
+  ATTN_ERR_BAD_SEQLENS = 5,  /* device: cu_seqlens contents inconsistent      */
+  ATTN_ERR_TIMEOUT = 6,      /* device: a bounded wait ran out                */
+  ATTN_ERR_CUDA = 7          /* a CUDA runtime or driver call failed          */
+} attn_status_t;
+
+typedef struct {
+  int32_t total_tokens; /* T                                                  */
+  int32_t num_seqs;     /* number of documents                              */
+  int32_t num_heads;    /* H                                                  */
+  int32_t head_dim;     /* d                                                  */
+  int32_t max_seqlen;   /* upper bound of every document length (dense: N)  */
+} attn_shape_t;
+
+/* Bytes of device workspace attn_fwd needs for this shape and dtype.  The
+ * workspace holds the error word, the work list of the schedule-build step
+ * and, for ATTN_MXFP8, the quantised operands.  Returns 0 for an invalid
+ * shape.  Layout (for tests and tools): int32 error word at byte 0, int32
+ * work-list length at byte 4, int32 [n][4] work list at byte 256, one entry
+ * (doc_start, doc_len, pair_index, cost) per pair of 128-row query tiles,
+ * sorted by cost, largest first, ties in document then pair order. */
+size_t attn_workspace_size(const attn_shape_t* shape, attn_dtype_t dtype);
+
+/* Exact attention forward.  q, k, v: bf16 [T, H, d]; out: bf16 [T, H, d];
+ * lse: fp32 [H, T] (natural log, scaled-score units); causal: 0 or 1;
+ * scale: the factor applied to q.k (1/sqrt(d) for standard attention).
+ * Launches the schedule-build kernel, the MXFP8 quantisation kernel (dtype
+ * ATTN_MXFP8 only) and the attention kernel on `stream`. */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                       void* out, float* lse, int causal, float scale, attn_dtype_t dtype,
+                       void* stream, const attn_shape_t* shape, void* workspace,
+                       size_t workspace_bytes);
+
+/* The MXFP8 quantisation pre-pass on its own (FLAMIA section "FLAMIA
+ * Mimarisi ve Temel Tasarım İlkeleri": quantisation fused into the
+ * kernels).  x: bf16 [rows, cols] device, cols a multiple of 32 and of 8;
+ * codes: uint8 [rows, cols] E4M3; scales: uint8 [rows, cols / 32] E8M0
+ * (code c means 2^(c - 127)).  Scale rule: the smallest power of two that
+ * maps the block's largest magnitude to at most 448; code clamped to
+ * [0, 254]; an all-zero block gets 127.  Elements: x / 2^(c-127) rounded to
+ * nearest E4M3 (ties to even, saturating at 448).  Asynchronous. */
+attn_status_t attn_quantize_mxfp8(const void* x, uint8_t* codes, uint8_t* scales, int64_t rows,
+                                  int32_t cols, void* stream);
+
+/* Synchronises `stream`, then reads the workspace's error word into
+ * *device_status and clears it.  The word holds the outcome of the most
+ * recent attn_fwd on this workspace (each call resets it when it starts):
+ * ATTN_OK, ATTN_ERR_BAD_SEQLENS or ATTN_ERR_TIMEOUT.  Returns ATTN_ERR_CUDA
+ * if the copy fails. */
+attn_status_t attn_get_device_error(const void* workspace, void* stream,
+                                    int32_t* device_status);
+
+/* Static, human-readable name of a status code. */
+const char* attn_status_string(attn_status_t status);
+
+/* ATTN_ABI_VERSION of the built library. */
+int32_t attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_TILED_ATTENTION_ATTN_H */

@@ -1,0 +1,87 @@
+"""The C-ABI library: it loads, exports every function include/attn.h
+declares, and its host-only paths (argument checks, sizes, strings) behave
+as documented.  No kernel is launched, so these run without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_tiled_attention_39_b200 import attn as A
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(attn_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from exact_tiled_attention_39_b200 import build
+    build.build()
+    return A.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared_functions()
+    assert "attn_fwd" in declared and "attn_quantize_mxfp8" in declared
+    for name in declared:
+        assert hasattr(L, name), f"libattn.so does not export {name}"
+    assert set(A.EXPORTED_SYMBOLS) <= set(declared)
+
+
+def test_version_and_strings(L):
+    assert L.attn_abi_version() == 1
+    assert A.status_string(0) == "ATTN_OK"
+    assert A.status_string(5) == "ATTN_ERR_BAD_SEQLENS"
+    assert A.status_string(6) == "ATTN_ERR_TIMEOUT"
+
+
+def test_workspace_size(L):
+    s = A.Shape(16384, 7, 32, 128, 4096)
+    n_bf16 = A.workspace_size(s, A.ATTN_BF16)
+    n_mx = A.workspace_size(s, A.ATTN_MXFP8)
+    max_entries = 16384 // 256 + 7 + 1
+    assert n_bf16 >= 256 + 2 * 16 * max_entries
+    assert n_mx >= n_bf16 + 3 * 16384 * 32 * 128 + 3 * 16384 * 32 * 4
+    assert A.workspace_size(A.Shape(16, 1, 1, 96, 16)) == 0       # d unsupported
+    assert A.workspace_size(A.Shape(-1, 1, 1, 64, 16)) == 0
+
+
+def _fwd(L, shape, ptrs=(16, 16, 16, 16, 16), ws=16, ws_bytes=1 << 20, scale=0.125, causal=1,
+         dtype=0, cu=None):
+    s = shape.c() if shape is not None else None
+    q, k, v, o, l = (ctypes.c_void_p(p) if p else None for p in ptrs)
+    return L.attn_fwd(q, k, v, cu, o, l, causal, scale, dtype, None,
+                      ctypes.byref(s) if s is not None else None,
+                      ctypes.c_void_p(ws) if ws else None, ws_bytes)
+
+
+def test_host_checks_return_before_launch(L):
+    ok = A.Shape(256, 1, 2, 64, 256)
+    assert _fwd(L, None) == 1                                   # NULL shape
+    assert _fwd(L, A.Shape(256, 1, 2, 96, 256)) == 2            # d unsupported
+    assert _fwd(L, ok, dtype=7) == 2
+    assert _fwd(L, ok, scale=0.0) == 1
+    assert _fwd(L, ok, scale=float("nan")) == 1
+    assert _fwd(L, ok, causal=2) == 1
+    assert _fwd(L, A.Shape(256, 2, 2, 64, 100)) == 1            # dense: T != B*N
+    assert _fwd(L, ok, ptrs=(16, 16, 0, 16, 16)) == 1           # NULL v
+    assert _fwd(L, ok, ptrs=(16, 24, 16, 16, 16)) == 3          # misaligned k
+    assert _fwd(L, ok, ws=0) == 4
+    assert _fwd(L, ok, ws_bytes=8) == 4
+    assert _fwd(L, A.Shape(0, 0, 2, 64, 0), ptrs=(0, 0, 0, 0, 0)) == 0   # T == 0: no-op
+
+
+def test_quantize_host_checks(L):
+    assert L.attn_quantize_mxfp8(None, None, None, 4, 48, None) == 1     # cols % 32
+    assert L.attn_quantize_mxfp8(None, None, None, 0, 64, None) == 0     # empty: no-op
+    assert L.attn_quantize_mxfp8(ctypes.c_void_p(16), ctypes.c_void_p(8), ctypes.c_void_p(16),
+                                 4, 64, None) == 3
