@@ -166,3 +166,31 @@ def attn_get_device_error(workspace, stream=None) -> int:
     if rc != 0:
         raise AttnError(rc, "attn_get_device_error")
     return int(v.value)
+
+
+def attn_fwd_noalloc(q, k, v, cu_seqlens, out, lse, causal: bool, scale: float, stream=None,
+                     max_seqlen: int | None = None, num_seqs: int | None = None) -> None:
+    """The bf16 forward through ``attn_fwd_noalloc``: no workspace is passed
+    and nothing is allocated (the library's fixed 1 MiB device scratch is
+    used).  For callers that cannot allocate device memory; calls that
+    overlap on the GPU race on the shared scratch."""
+    L = lib()
+    fn = L.attn_fwd_noalloc
+    vp = ctypes.c_void_p
+    fn.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_float, vp,
+                   ctypes.POINTER(_Shape)]
+    fn.restype = ctypes.c_int
+    T, H, d = q.shape
+    if cu_seqlens is not None:
+        ns = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens (no host sync is done)")
+    else:
+        ns = num_seqs if num_seqs is not None else 1
+        if max_seqlen is None:
+            max_seqlen = T // max(ns, 1)
+    s = Shape(T, ns, H, d, int(max_seqlen)).c()
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(out), _ptr(lse),
+            int(bool(causal)), float(scale), _stream_handle(stream, q.device), ctypes.byref(s))
+    if rc != 0:
+        raise AttnError(rc, "attn_fwd_noalloc")

@@ -245,3 +245,52 @@ attn_status_t attn_get_device_error(const void* workspace, void* stream, int32_t
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// attn_fwd_noalloc: the bf16 forward for callers that cannot allocate device
+// memory (see include/attn.h).  Its scratch - the error word and the two
+// work lists the schedule-build kernel writes and the attention kernel reads
+// - is this fixed array, part of the library's device image: every GPU that
+// loads the library holds it until the process exits.  All calls share it.
+// ---------------------------------------------------------------------------
+namespace attn {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array, looked up once per device with that device
+// current.  In host code `g_noalloc_scratch` names a host-side stand-in, not
+// device memory, so it is never passed to a kernel directly.
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+}  // namespace
+}  // namespace attn
+
+extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                          const int32_t* cu_seqlens, void* out, float* lse,
+                                          int causal, float scale, void* stream,
+                                          const attn_shape_t* shape) {
+  const attn_status_t st = check_shape(shape);
+  if (st != ATTN_OK) return st;
+  // Reject problems whose work lists do not fit the fixed scratch.
+  if (ws_layout(*shape, ATTN_BF16).total > kNoAllocScratchBytes) return ATTN_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return ATTN_ERR_CUDA;
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  // The schedule-build kernel rewrites the error word, the list length and
+  // both lists on every call, so nothing left by an earlier call is read.
+  return attn_fwd(q, k, v, cu_seqlens, out, lse, causal, scale, ATTN_BF16, stream, shape,
+                  scratch, kNoAllocScratchBytes);
+}

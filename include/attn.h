@@ -107,6 +107,34 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
                        void* stream, const attn_shape_t* shape, void* workspace,
                        size_t workspace_bytes);
 
+/* attn_fwd for callers that cannot allocate device memory: a plugin or
+ * custom operator that its host application hands only input and output
+ * buffers, code running under a device-memory budget fixed up front by a
+ * serving framework, or a latency-critical path that cannot afford the
+ * implicit device synchronisation of cudaMalloc.  The pages have no
+ * counterpart: this is an interface convenience, not part of the method.
+ *
+ * Same arguments and results as attn_fwd with dtype ATTN_BF16, minus the
+ * workspace: its scratch (error word and work lists) is a 1 MiB array
+ * inside the library's device image, which every GPU that loads the library
+ * holds until the process exits.  Problems whose work lists need more
+ * (total_tokens / 256 + num_seqs > 32751) are rejected with
+ * ATTN_ERR_WORKSPACE before anything is launched.  Nothing is allocated: no
+ * cudaMalloc, cudaFree or allocating library routine is called.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls share the one array, and every call
+ * rewrites what it reads (the error word is reset, the lists rebuilt), so
+ * sequential calls are independent; calls that overlap on the GPU (other
+ * streams, other host threads) race on the array and must be serialised by
+ * the caller.  Device-side faults (bad cu_seqlens contents, a wait running
+ * out) leave out and lse unwritten as with attn_fwd; their error word is in
+ * the array and is not readable through this ABI. */
+attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                               const int32_t* cu_seqlens, void* out, float* lse, int causal,
+                               float scale, void* stream, const attn_shape_t* shape);
+
 /* The MXFP8 quantisation pre-pass on its own (FLAMIA section "FLAMIA
  * Mimarisi ve Temel Tasarım İlkeleri": quantisation fused into the
  * kernels).  x: bf16 [rows, cols] device, cols a multiple of 32 and of 8;
