@@ -221,12 +221,27 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   fp.timeout_ns = kWaitTimeoutNs;
   const int64_t max_units = wl.max_entries * s.num_heads;
   const int grid = static_cast<int>(max_units < info.num_sms ? max_units : info.num_sms);
+  // Programmatic dependent launch: the attention kernel's prologue (barrier
+  // set-up, TMEM allocation, tensor-map prefetch) overlaps the schedule
+  // kernel; it waits for the work list with griddepcontrol.wait.
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kFwdThreads);
+  cfg.stream = strm;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   if (s.head_dim == 128) {
-    attn_fwd_bf16_kernel<128><<<grid, 384, FwdLayout<128>::kAllocBytes, strm>>>(tq, tk, tv, fp);
+    cfg.dynamicSmemBytes = FwdLayout<128>::kAllocBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_bf16_kernel<128>, tq, tk, tv, fp);
   } else {
-    attn_fwd_bf16_kernel<64><<<grid, 384, FwdLayout<64>::kAllocBytes, strm>>>(tq, tk, tv, fp);
+    cfg.dynamicSmemBytes = FwdLayout<64>::kAllocBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_bf16_kernel<64>, tq, tk, tv, fp);
   }
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 attn_status_t attn_get_device_error(const void* workspace, void* stream, int32_t* device_status) {

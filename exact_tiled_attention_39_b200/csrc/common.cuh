@@ -15,6 +15,7 @@ constexpr int kRowsPerUnit = kBlockM * kTilesPerUnit;
 // Workspace layout: a 256-byte header, then the work list.
 constexpr size_t kWsErrorOffset = 0;     // int32 error word (attn_status_t)
 constexpr size_t kWsCountOffset = 4;     // int32 number of work-list entries
+constexpr size_t kWsUnitCounterOffset = 8;   // int32 dynamic unit counter (reset per call)
 constexpr size_t kWsListOffset = 256;    // int4 entries
 constexpr size_t kWsAlign = 256;
 

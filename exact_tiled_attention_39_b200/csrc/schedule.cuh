@@ -17,6 +17,7 @@
 #include <cstdint>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace attn {
 
@@ -70,8 +71,16 @@ build_schedule_kernel(const int32_t* __restrict__ cu, int num_seqs, int total_to
   __shared__ int chunk_total;
   const int tid = threadIdx.x, nt = blockDim.x;
 
-  // 0. the error word reports the most recent call only
-  if (tid == 0) ws_header[kWsErrorOffset / 4] = 0;
+  // The attention kernel queued behind this one may start its prologue now;
+  // it reads the work list only after this grid has completed.
+  ptx::grid_launch_dependents();
+
+  // 0. the error word reports the most recent call only; the attention
+  // kernel's unit counter starts from zero
+  if (tid == 0) {
+    ws_header[kWsErrorOffset / 4] = 0;
+    ws_header[kWsUnitCounterOffset / 4] = 0;
+  }
 
   // 1. validate the document offsets
   int bad = 0;

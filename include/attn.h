@@ -72,7 +72,9 @@ typedef enum {
 typedef enum {
   ATTN_OK = 0,
   ATTN_ERR_INVALID_ARG = 1,  /* NULL pointer, negative size, bad scale, ...   */
-  ATTN_ERR_UNSUPPORTED = 2,  /* head_dim or dtype not supported               */
+  ATTN_ERR_UNSUPPORTED = 2,  /* head_dim or dtype not supported (also recorded
+                                by a kernel that finds its shared memory
+                                misaligned; never observed)                    */
   ATTN_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned              */
   ATTN_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than required       */
   ATTN_ERR_BAD_SEQLENS = 5,  /* device: cu_seqlens contents inconsistent      */
