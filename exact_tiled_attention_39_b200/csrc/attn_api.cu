@@ -45,6 +45,8 @@ int64_t sort_capacity_for(int64_t max_entries) {
 
 struct WsLayout {
   size_t sorted_off, unsorted_off, mx_off, total;
+  // MXFP8: per operand (q, k, v) E4M3 codes, E8M0 scales, bf16 dequantised copy
+  size_t codes_off[3], scales_off[3], deq_off[3];
   int64_t max_entries;
 };
 
@@ -57,7 +59,14 @@ WsLayout ws_layout(const attn_shape_t& s, attn_dtype_t dtype) {
   w.total = w.mx_off;
   if (dtype == ATTN_MXFP8) {
     const size_t elems = static_cast<size_t>(s.total_tokens) * s.num_heads * s.head_dim;
-    w.total += 3 * align_up(elems, kWsAlign) + 3 * align_up(elems / 32, kWsAlign);
+    for (int i = 0; i < 3; ++i) {
+      w.codes_off[i] = w.total;
+      w.total = align_up(w.total + elems, kWsAlign);
+      w.scales_off[i] = w.total;
+      w.total = align_up(w.total + elems / 32, kWsAlign);
+      w.deq_off[i] = w.total;
+      w.total = align_up(w.total + 2 * elems, kWsAlign);
+    }
   }
   return w;
 }
@@ -161,7 +170,7 @@ attn_status_t attn_quantize_mxfp8(const void* x, uint8_t* codes, uint8_t* scales
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   quantize_mxfp8_kernel<<<static_cast<unsigned>(grid), threads, 0,
                           static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(x), reinterpret_cast<uint4*>(codes), scales, n_blocks);
+      static_cast<const uint4*>(x), reinterpret_cast<uint4*>(codes), scales, nullptr, n_blocks);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -185,7 +194,6 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   const WsLayout wl = ws_layout(s, dtype);
   if (workspace == nullptr || workspace_bytes < wl.total) return ATTN_ERR_WORKSPACE;
   if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
-  if (dtype == ATTN_MXFP8) return ATTN_ERR_UNSUPPORTED;
 
   int dev = 0;
   DeviceInfo info;
@@ -202,7 +210,25 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
       static_cast<int>(cap));
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
-  // 2. attention
+  // 2. MXFP8: quantise q, k, v (E4M3 + one E8M0 scale per token, head and 32
+  // head-dim elements) and run the products on the exact dequantised values.
+  if (dtype == ATTN_MXFP8) {
+    const void* src[3] = {q, k, v};
+    const long long n_blocks =
+        static_cast<long long>(s.total_tokens) * s.num_heads * (s.head_dim / 32);
+    const unsigned qgrid = static_cast<unsigned>((n_blocks + 255) / 256);
+    for (int i = 0; i < 3; ++i) {
+      quantize_mxfp8_kernel<<<qgrid, 256, 0, strm>>>(
+          static_cast<const uint4*>(src[i]), reinterpret_cast<uint4*>(ws + wl.codes_off[i]),
+          ws + wl.scales_off[i], reinterpret_cast<uint4*>(ws + wl.deq_off[i]), n_blocks);
+    }
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    q = ws + wl.deq_off[0];
+    k = ws + wl.deq_off[1];
+    v = ws + wl.deq_off[2];
+  }
+
+  // 3. attention
   CUtensorMap tq, tk, tv;
   if (!encode_qkv_map(&tq, q, s.total_tokens, s.num_heads, s.head_dim) ||
       !encode_qkv_map(&tk, k, s.total_tokens, s.num_heads, s.head_dim) ||

@@ -418,7 +418,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
             const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[2 * k], s[2 * k + 1]), c2, nb2);
             float x0, x1, p0, p1;
             ptx::f2_unpack(x, x0, x1);
-            if (kPolyPairPeriod > 0 && k % kPolyPairPeriod == kPolyPairPeriod - 1) {
+            if (kPolyPairPeriod > 0 && k % (kPolyPairPeriod > 0 ? kPolyPairPeriod : 1) == kPolyPairPeriod - 1) {
               exp2_poly_pair(x0, x1, p0, p1);
             } else {
               p0 = ptx::ex2_approx(x0);

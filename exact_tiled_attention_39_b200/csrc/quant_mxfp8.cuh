@@ -18,6 +18,8 @@
 //
 // HBM-bound: each thread reads one 64-byte block and writes 32 + 1 bytes.
 #pragma once
+#include <cuda_fp16.h>
+
 #include <cstdint>
 
 namespace attn {
@@ -49,10 +51,21 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// One thread per 32-element block; n_blocks = rows * cols / 32.
+// E4M3 pair -> two fp32 (exact: through f16, which holds every E4M3 value).
+__device__ __forceinline__ void e4m3x2_to_f32(uint16_t v, float& lo, float& hi) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
+  lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+  hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+}
+
+// One thread per 32-element block; n_blocks = rows * cols / 32.  When `deq`
+// is not null the exact dequantised values (E4M3 value * 2^(code - 127)) are
+// also written as bf16: a 4-bit significand times a power of two is exact in
+// bf16 over the whole range the scale rule produces.
 __global__ void __launch_bounds__(256)
 quantize_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ codes,
-                      uint8_t* __restrict__ scales, long long n_blocks) {
+                      uint8_t* __restrict__ scales, uint4* __restrict__ deq, long long n_blocks) {
   const long long b = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (b >= n_blocks) return;
   uint4 v[4];
@@ -77,6 +90,21 @@ quantize_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ codes,
   codes[2 * b] = make_uint4(out[0], out[1], out[2], out[3]);
   codes[2 * b + 1] = make_uint4(out[4], out[5], out[6], out[7]);
   scales[b] = static_cast<uint8_t>(code);
+  if (deq != nullptr) {
+    // 2^(code - 127); code 0 needs 2^-127 (subnormal)
+    const float mul = code == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(code << 23);
+    uint32_t y[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float f0, f1, f2, f3;
+      e4m3x2_to_f32(static_cast<uint16_t>(out[i] & 0xFFFFu), f0, f1);
+      e4m3x2_to_f32(static_cast<uint16_t>(out[i] >> 16), f2, f3);
+      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(y[2 * i]) : "f"(f1 * mul), "f"(f0 * mul));
+      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(y[2 * i + 1]) : "f"(f3 * mul), "f"(f2 * mul));
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) deq[4 * b + i] = make_uint4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+  }
 }
 
 }  // namespace attn
