@@ -9,7 +9,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "attn_fwd_bf16.cuh"
+#include "attn_fwd_sm100.cuh"
 #include "common.cuh"
 #include "quant_mxfp8.cuh"
 #include "schedule.cuh"
@@ -99,11 +99,15 @@ attn_status_t device_info(int* dev_out, DeviceInfo* info) {
   if (!d.ready) {
     if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    if (cudaFuncSetAttribute(attn_fwd_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FwdLayout<64>::kAllocBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_bf16_kernel<128>,
+    if (cudaFuncSetAttribute(attn_fwd_kernel<64, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FwdLayout<128>::kAllocBytes) != cudaSuccess ||
+                             FwdLayout<64, false>::kBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<128, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FwdLayout<128, false>::kBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<128, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FwdLayout<128, true>::kBytes) != cudaSuccess ||
         cudaFuncSetAttribute(build_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSortCapacityMax * 8) != cudaSuccess)
       return ATTN_ERR_CUDA;
@@ -114,17 +118,20 @@ attn_status_t device_info(int* dev_out, DeviceInfo* info) {
   return ATTN_OK;
 }
 
-// 3-D map over a [T, H, d] bf16 tensor: box = 64 head-dim elements (128 B,
-// the swizzle span) x 1 head x 128 tokens, 128-byte swizzle, zero fill.
-bool encode_qkv_map(CUtensorMap* m, const void* base, int T, int H, int d) {
+// 3-D map over a [T, H, d] tensor of `elem` bytes per element: box = 128
+// bytes of head dim (the swizzle span) x 1 head x 128 tokens, 128-byte
+// swizzle, zero fill outside the tensor.
+bool encode_qkv_map(CUtensorMap* m, const void* base, int T, int H, int d, int elem) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(T)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(H) * d * 2};
-  const cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kBlockM)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem,
+                                 static_cast<cuuint64_t>(H) * d * elem};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), 1,
+                             static_cast<cuuint32_t>(kBlockM)};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return g_encode(m, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                  3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -211,7 +218,11 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
   // 2. MXFP8: quantise q, k, v (E4M3 + one E8M0 scale per token, head and 32
-  // head-dim elements) and run the products on the exact dequantised values.
+  // head-dim elements).  With d = 128 the score product runs block-scaled on
+  // the E4M3 codes of q and k, and P V on the exact bf16 dequantisation of v;
+  // with d = 64 all three products run on the dequantised values.
+  const bool fp8_kernel = dtype == ATTN_MXFP8 && s.head_dim == 128;
+  const void* qk_src[2] = {q, k};
   if (dtype == ATTN_MXFP8) {
     const void* src[3] = {q, k, v};
     const long long n_blocks =
@@ -223,16 +234,16 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
           ws + wl.scales_off[i], reinterpret_cast<uint4*>(ws + wl.deq_off[i]), n_blocks);
     }
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-    q = ws + wl.deq_off[0];
-    k = ws + wl.deq_off[1];
+    for (int i = 0; i < 2; ++i) qk_src[i] = ws + (fp8_kernel ? wl.codes_off[i] : wl.deq_off[i]);
     v = ws + wl.deq_off[2];
   }
 
   // 3. attention
+  const int qk_elem = fp8_kernel ? 1 : 2;
   CUtensorMap tq, tk, tv;
-  if (!encode_qkv_map(&tq, q, s.total_tokens, s.num_heads, s.head_dim) ||
-      !encode_qkv_map(&tk, k, s.total_tokens, s.num_heads, s.head_dim) ||
-      !encode_qkv_map(&tv, v, s.total_tokens, s.num_heads, s.head_dim))
+  if (!encode_qkv_map(&tq, qk_src[0], s.total_tokens, s.num_heads, s.head_dim, qk_elem) ||
+      !encode_qkv_map(&tk, qk_src[1], s.total_tokens, s.num_heads, s.head_dim, qk_elem) ||
+      !encode_qkv_map(&tv, v, s.total_tokens, s.num_heads, s.head_dim, 2))
     return ATTN_ERR_CUDA;
   FwdParams fp;
   fp.out = out;
@@ -240,6 +251,8 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   fp.ws_header = header;
   fp.work = reinterpret_cast<const int4*>(ws + wl.sorted_off);
   fp.err = header + kWsErrorOffset / 4;
+  fp.q_scales = fp8_kernel ? reinterpret_cast<const uint32_t*>(ws + wl.scales_off[0]) : nullptr;
+  fp.k_scales = fp8_kernel ? reinterpret_cast<const uint32_t*>(ws + wl.scales_off[1]) : nullptr;
   fp.total_tokens = s.total_tokens;
   fp.num_heads = s.num_heads;
   fp.causal = causal;
@@ -260,12 +273,15 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (s.head_dim == 128) {
-    cfg.dynamicSmemBytes = FwdLayout<128>::kAllocBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_bf16_kernel<128>, tq, tk, tv, fp);
+  if (fp8_kernel) {
+    cfg.dynamicSmemBytes = FwdLayout<128, true>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, true>, tq, tk, tv, fp);
+  } else if (s.head_dim == 128) {
+    cfg.dynamicSmemBytes = FwdLayout<128, false>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, false>, tq, tk, tv, fp);
   } else {
-    cfg.dynamicSmemBytes = FwdLayout<64>::kAllocBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_bf16_kernel<64>, tq, tk, tv, fp);
+    cfg.dynamicSmemBytes = FwdLayout<64, false>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<64, false>, tq, tk, tv, fp);
   }
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -1,0 +1,753 @@
+// Exact attention forward for sm_100a: persistent, warp-specialised,
+// TMA + tcgen05 + TMEM; bf16 operands, or MXFP8 (E4M3 with E8M0 block scales)
+// for the score product.
+//
+// The method ("FlashAttention và IO" (aihero.vn), sections "Tiling giữ công
+// việc ở gần nơi tính" and "Softmax qua nhiều khối cần thống kê chạy"):
+// Q, K and V are cut into tiles held on chip; for each query row the kernel
+// keeps the running maximum m, the normaliser l and the weighted sum u (the
+// output accumulator O), multiplies the old part by exp(m - m_new) when a new
+// key tile raises the maximum, and writes u / l and the log-sum-exp at the
+// end.  Scores and probabilities never leave the SM.
+//
+// Loop order and roles follow "FlashAttention, pelatihan multi-GPU, dan
+// kuantisasi bobot" (section 1): outer loop over query blocks, inner over
+// key/value blocks; a producer issues asynchronous tile copies while other
+// warps run the products and the softmax.  The MXFP8 variant follows
+// "FLAMIA: Blackwell Üzerinde Hızlı ve Nedensel Olarak Güvenli Eğitim İçin
+// Flash Mikro-Ölçeklemeli Dikkat Mekanizması" (section "FLAMIA Mimarisi ve
+// Temel Tasarım İlkeleri"): block-scaled low-precision products whose scales
+// (one per token, head and 32 head-dim elements) never span two tokens.
+//
+// A work unit is one 128-row query tile of one document and head.  On
+// sm_100a (384 threads, registers re-split per warpgroup with setmaxnreg):
+//
+//   warps 0..3    softmax (232 registers): one thread per query row reads its
+//                 score row from TMEM, masks, updates m and l, writes P (bf16)
+//                 back over the scores, and rescales O when its maximum grew
+//                 by more than 2^8 (lazy rescale).
+//   warps 4..7    epilogue (120 registers): O / l to bf16 and the log-sum-exp.
+//   warp 8        producer (152 registers): claims units, TMA loads of Q and of
+//                 K_j, V_j into a ring of shared-memory slots; for MXFP8 the
+//                 whole warp also stages the E8M0 scale blocks.
+//   warp 9        MMA issuer (one thread): S = Q K_j^T into one of two TMEM
+//                 score buffers, O += P V_j with P read from TMEM.
+//   warps 10..11  idle.
+//
+// The score buffers alternate between key steps, so while the softmax works
+// on step j the tensor core computes P_{j-1} V_{j-1} and S_{j+1}.
+//
+// TMEM (512 columns, lane = query row): S buffers at columns 0 and 128 (P
+// overwrites the first 64 columns of its buffer), O at 256; for MXFP8 the
+// scale factors of Q at 384 and of the current K tile at 388 / 392.
+#pragma once
+#include <cuda.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace attn {
+
+struct FwdParams {
+  void* out;                 // bf16 [T, H, D]
+  float* lse;                // fp32 [H, T]
+  const int32_t* ws_header;  // error word, work-list length, unit counter
+  const int4* work;          // work list
+  int32_t* err;              // error word (device)
+  const uint32_t* q_scales;  // MXFP8: E8M0 words [T, H] (4 scales per word)
+  const uint32_t* k_scales;
+  int total_tokens;
+  int num_heads;
+  int causal;
+  float scale_log2;          // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+constexpr int kFwdThreads = 384;
+// Registers per thread at launch: 65536 / 384 rounded down to a multiple of 8.
+// Each warpgroup moves once, at the start of its role, and keeps that count:
+// a warpgroup that lowered its count and raised it again could take back
+// registers before the softmax warpgroup's increase is served.
+constexpr uint32_t kRegsEntry = 168;
+constexpr uint32_t kRegsSoftmax = 232, kRegsEpilogue = 120, kRegsOther = 152;
+static_assert(kRegsSoftmax + kRegsEpilogue + kRegsOther == 3 * kRegsEntry,
+              "register split must use exactly the registers the CTA is launched with");
+
+constexpr int kUnitSlots = 4;
+constexpr int kUnitConsumers = 1 + 4 + 4;   // MMA thread + softmax warps + epilogue warps
+
+// Exponentials: most run on the MUFU unit (ex2.approx); pairs of keys with
+// index k % period == period - 1 run on the FMA pipe instead, as 2^x =
+// 2^floor(x) * p(frac(x)) with the polynomial below (0 = MUFU only).  The MUFU
+// unit alone cannot keep up with the tensor core (16 exponentials per SM and
+// cycle against 128 x 128 scores per 128 x 128 x D product pair).
+#ifndef ATTN_POLY_PAIR_PERIOD
+#define ATTN_POLY_PAIR_PERIOD 0
+#endif
+constexpr int kPolyPairPeriod = ATTN_POLY_PAIR_PERIOD;
+
+// 2^f on [0, 1): 1 + f (c1 + f (c2 + f c3)), a minimax fit of the relative
+// error (max 8.6e-5) made by csrc/fit_exp2_poly.py; p(0) = 1 exactly.
+constexpr float kExp2C1 = 6.951168180e-01f;
+constexpr float kExp2C2 = 2.276448607e-01f;
+constexpr float kExp2C3 = 7.706713676e-02f;
+
+template <int D, bool kFp8>
+struct FwdLayout {
+  static_assert(D == 64 || D == 128, "head dim 64 or 128");
+  static_assert(!kFp8 || D == 128, "the MXFP8 kernel is built for head dim 128");
+  static constexpr int kQKChunks = kFp8 ? 1 : D / 64;        // 128-byte chunks per Q/K row
+  static constexpr int kVChunks = D / 64;                     // V is bf16
+  static constexpr int kChunkBytes = kBlockM * 128;           // 128 rows x 128 bytes
+  static constexpr int kQBytes = kQKChunks * kChunkBytes;
+  static constexpr int kKBytes = kQKChunks * kChunkBytes;
+  static constexpr int kVBytes = kVChunks * kChunkBytes;
+  static constexpr int kSfBytes = 512;                        // 128 rows x 4 scale bytes
+  static constexpr int kSlotBytes = kVBytes;                  // a V tile, or a K tile + scales
+  static_assert(kKBytes + (kFp8 ? kSfBytes : 0) <= kSlotBytes, "K tile must fit a slot");
+  static constexpr int kQOff = 0;
+  static constexpr int kSfaOff = kQBytes;                     // MXFP8 only
+  static constexpr int kRingOff = ((kQBytes + (kFp8 ? kSfBytes : 0)) + 1023) / 1024 * 1024;
+  static constexpr int kReserve = 4096;                       // stats, barriers, ring of units
+  static constexpr int kStagesFit = (232448 - kRingOff - kReserve) / kSlotBytes;
+  static constexpr int kStages = kStagesFit > 10 ? 10 : kStagesFit;
+  static constexpr int kStatsOff = kRingOff + kStages * kSlotBytes;   // float [2][128]
+  static constexpr int kBarOff = kStatsOff + 2 * kBlockM * 4;
+  static constexpr int kQFull = 0, kQEmpty = 1;
+  static constexpr int kKVFull = 2;                           // + stage
+  static constexpr int kKVEmpty = kKVFull + kStages;          // + stage
+  static constexpr int kSFull = kKVEmpty + kStages;           // + buffer
+  static constexpr int kPFull = kSFull + 2;                   // + buffer
+  static constexpr int kOFull = kPFull + 2;
+  static constexpr int kOEmpty = kOFull + 1;
+  static constexpr int kStFull = kOEmpty + 1;
+  static constexpr int kStEmpty = kStFull + 1;
+  static constexpr int kDrain = kStEmpty + 1;
+  static constexpr int kUnitFull = kDrain + 1;                // + slot
+  static constexpr int kUnitEmpty = kUnitFull + kUnitSlots;   // + slot
+  static constexpr int kNumBars = kUnitEmpty + kUnitSlots;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;     // tmem base, abort flag
+  static constexpr int kUnitOff = kMiscOff + 16;              // int32 [kUnitSlots]
+  static constexpr int kBytes = kUnitOff + 4 * kUnitSlots;
+  static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
+  static_assert(kBytes - kStatsOff <= kReserve, "reserve too small");
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmemO = 256, kTmemSfa = 384, kTmemSfb = 388;
+};
+
+// Bounded waits.  A wait gives up when the CTA's abort flag is raised or
+// after timeout_ns; the first thread to give up records ATTN_ERR_TIMEOUT.
+// They are inlined and take their control block by value: a real call with
+// a stack frame cannot be register-allocated inside a setmaxnreg region.
+struct WaitCtl {
+  volatile uint32_t* abort_flag;
+  int32_t* err;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ void raise_abort(WaitCtl c) {
+  if (*c.abort_flag == 0) {
+    *c.abort_flag = 1;
+    atomicCAS(c.err, 0, (int)ATTN_ERR_TIMEOUT);
+  }
+}
+
+// Single-thread bounded wait.
+__device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, WaitCtl c) {
+  if (ptx::mbar_test(bar, parity)) return true;
+  unsigned long long t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_test(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (*c.abort_flag) return false;
+      if (ptx::globaltimer_ns() - t0 > c.timeout_ns) {
+        raise_abort(c);
+        return false;
+      }
+    }
+  }
+}
+
+// Warp-uniform bounded wait: every lane probes; the warp leaves together.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, WaitCtl c) {
+  if (__all_sync(0xffffffffu, ptx::mbar_test(bar, parity))) return true;
+  unsigned long long t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (__all_sync(0xffffffffu, ptx::mbar_test(bar, parity))) return true;
+    if ((it & 63) == 0) {
+      bool give_up = *c.abort_flag != 0;
+      give_up |= ptx::globaltimer_ns() - t0 > c.timeout_ns;
+      if (__any_sync(0xffffffffu, give_up)) {
+        if (ptx::lane_id() == 0) raise_abort(c);
+        return false;
+      }
+    }
+  }
+}
+
+struct UnitInfo {
+  int doc_start, doc_len, qb, head, kv_tiles, n;   // n = key steps of this tile
+};
+
+__device__ __forceinline__ UnitInfo decode_unit(const int4* work, int u, int H, int causal) {
+  const int4 w = work[u / H];
+  UnitInfo r;
+  r.doc_start = w.x;
+  r.doc_len = w.y;
+  r.qb = w.z;
+  r.head = u % H;
+  r.kv_tiles = (w.y + kBlockN - 1) / kBlockN;
+  r.n = causal ? min(w.z + 1, r.kv_tiles) : r.kv_tiles;
+  return r;
+}
+
+// 2^x for a pair of x <= 8 on the FMA pipe.  x = j + f with j = floor(x)
+// (taken from adding 1.5 * 2^23 rounded down, which leaves j in the low
+// mantissa bits), 2^f from the polynomial, and j added to the exponent
+// field.  x is clamped at -127 first, where the result is exactly +0 (the
+// exponent field of p(0) = 1 cancels), so masked scores (-inf) give 0.
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
+  const uint64_t x = ptx::f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const float kMagic = 12582912.f;   // 1.5 * 2^23
+  const uint64_t t = ptx::f2_add_rm(x, ptx::f2_pack(kMagic, kMagic));
+  const uint64_t jf = ptx::f2_add(t, ptx::f2_pack(-kMagic, -kMagic));
+  const uint64_t f = ptx::f2_fma(jf, ptx::f2_pack(-1.f, -1.f), x);
+  uint64_t q = ptx::f2_fma(ptx::f2_pack(kExp2C3, kExp2C3), f, ptx::f2_pack(kExp2C2, kExp2C2));
+  q = ptx::f2_fma(q, f, ptx::f2_pack(kExp2C1, kExp2C1));
+  q = ptx::f2_fma(q, f, ptx::f2_pack(1.f, 1.f));
+  float q0, q1, t0, t1;
+  ptx::f2_unpack(q, q0, q1);
+  ptx::f2_unpack(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte block of E8M0 scales for
+// tcgen05.cp (K-major, no swizzle: 8-row core matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t sf_copy_desc(uint32_t saddr) {
+  return ptx::sdesc_join(ptx::sdesc_lo(saddr, 512), ((128u >> 4) & 0x3FFFu) | (1u << 14));
+}
+
+// Instruction descriptor for the block-scaled E4M3 x E4M3 product (fp32
+// accumulate, E8M0 scales, M = N = 128, K = 32); sf_id picks the scale byte
+// (the 32-element block) inside each 32-bit scale column.
+__host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t sf_id) {
+  return (sf_id << 4)                         // B scale id
+         | (0u << 7) | (0u << 10)             // A, B format: E4M3
+         | (static_cast<uint32_t>(kBlockN >> 3) << 17)
+         | (1u << 23)                         // scale format: E8M0
+         | (static_cast<uint32_t>(kBlockM >> 4) << 24)
+         | (sf_id << 29);                     // A scale id
+}
+
+__device__ __forceinline__ void mma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copy a 32-row x 128-bit block from shared memory to TMEM lanes 0..31 and
+// replicate it into the other three lane quarters.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int D, bool kFp8>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using Lay = FwdLayout<D, kFp8>;
+  // The kernel has no static shared memory, so the dynamic block starts at
+  // the CTA's (1024-byte aligned) shared window; the 128-byte swizzle needs
+  // that alignment.  Checked anyway: a misaligned base records an error and
+  // the CTA leaves before touching anything.
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = ptx::smem_addr(smem);
+  if ((sbase & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicCAS(p.err, 0, (int)ATTN_ERR_UNSUPPORTED);
+    return;
+  }
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  auto bar = [&](int i) -> uint32_t { return sbase + Lay::kBarOff + 8 * i; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
+  volatile uint32_t* abort_flag = tmem_holder + 1;
+  float* stats = reinterpret_cast<float*>(smem + Lay::kStatsOff);   // [lse2, 1/l_round][row]
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + Lay::kUnitOff);
+
+  constexpr int kWarpTma = 8, kWarpMma = 9;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar(Lay::kQFull), 1);
+    ptx::mbar_init(bar(Lay::kQEmpty), 1);
+    for (int s = 0; s < Lay::kStages; ++s) {
+      ptx::mbar_init(bar(Lay::kKVFull + s), 1);
+      ptx::mbar_init(bar(Lay::kKVEmpty + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(bar(Lay::kSFull + b), 1);
+      ptx::mbar_init(bar(Lay::kPFull + b), 4);    // one arrival per softmax warp
+    }
+    ptx::mbar_init(bar(Lay::kOFull), 1);
+    ptx::mbar_init(bar(Lay::kOEmpty), 4);         // one arrival per epilogue warp
+    ptx::mbar_init(bar(Lay::kStFull), 4);
+    ptx::mbar_init(bar(Lay::kStEmpty), 4);
+    ptx::mbar_init(bar(Lay::kDrain), 1);
+    for (int i = 0; i < kUnitSlots; ++i) {
+      ptx::mbar_init(bar(Lay::kUnitFull + i), 1);
+      ptx::mbar_init(bar(Lay::kUnitEmpty + i), kUnitConsumers);
+    }
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == kWarpTma && lane == 0) {
+    ptx::prefetch_tmap(&tm_q);
+    ptx::prefetch_tmap(&tm_k);
+    ptx::prefetch_tmap(&tm_v);
+  }
+  if (warp == kWarpMma) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_holder), Lay::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  // The work list is written by the schedule-build kernel launched just
+  // before; everything above overlapped with its tail.
+  ptx::grid_dependency_wait();
+
+  const WaitCtl ctl{abort_flag, p.err, p.timeout_ns};
+  const int H = p.num_heads;
+  const int causal = p.causal;
+  // Consumer side of the unit ring: the k-th unit of this CTA, or -1 when the
+  // work is exhausted (also -1 if the wait gave up; `ok` says which).
+  auto next_unit_warp = [&](uint32_t k, bool& ok) -> int {
+    const uint32_t slot = k % kUnitSlots;
+    if (!(ok = wait_warp(bar(Lay::kUnitFull + slot), (k / kUnitSlots) & 1, ctl))) return -1;
+    const int u = unit_ring[slot];
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(bar(Lay::kUnitEmpty + slot));
+    return u;
+  };
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ softmax
+    ptx::regs_increase<kRegsSoftmax>();
+    const int r = warp * 32 + lane;               // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t t_o = tmem + lane_off + Lay::kTmemO;
+    const float c = p.scale_log2;
+    const uint64_t c2 = ptx::f2_pack(c, c);
+    uint32_t g = 0, st_cnt = 0;                   // global key step, units handed over
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      const int u = next_unit_warp(k, ok);
+      if (u < 0) break;
+      const UnitInfo ui = decode_unit(p.work, u, H, causal);
+      float m_used = -INFINITY;   // running maximum in log2 units
+      float l = 0.f;              // sum of the weights
+      float l_round = 0.f;        // sum of the weights as rounded to bf16
+      for (int j = 0; j < ui.n; ++j, ++g) {
+        const uint32_t buf = g & 1;
+        const uint32_t t_s = tmem + lane_off + buf * 128;
+        if (!(ok = wait_warp(bar(Lay::kSFull + buf), (g >> 1) & 1, ctl))) break;
+        ptx::tc_fence_after();
+        uint32_t sa[64], sb[64];
+        ptx::tmem_ld_x64(t_s, sa);
+        ptx::tmem_ld_x64(t_s + 64, sb);
+        float s[128];
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          s[q] = __uint_as_float(sa[q]);
+          s[64 + q] = __uint_as_float(sb[q]);
+        }
+        const bool diag = causal && j == ui.qb;
+        if (diag || (j + 1) * kBlockN > ui.doc_len) {
+          int limit = ui.doc_len - j * kBlockN;
+          if (diag) limit = min(limit, r + 1);
+#pragma unroll
+          for (int q = 0; q < 128; ++q)
+            if (q >= limit) s[q] = -INFINITY;
+        }
+        // Row maximum of the tile (8 independent chains).
+        auto tile_max = [&]() -> float {
+          float mx[8];
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx[a] = fmaxf(s[2 * a], s[2 * a + 1]);
+#pragma unroll
+          for (int q = 16; q < 128; q += 16)
+#pragma unroll
+            for (int a = 0; a < 8; ++a) mx[a] = ptx::fmax3(mx[a], s[q + 2 * a], s[q + 2 * a + 1]);
+          return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        };
+        // Weights are rounded to bf16 for the P V product.  Two normalisers:
+        // l_round sums the rounded weights, so O / l_round is an exact convex
+        // combination of the values with the weights actually used (no bias
+        // from the rounding, which matters when one key dominates a row);
+        // l sums the unrounded weights and gives the log-sum-exp.
+        // exp_pass: P = 2^(s c - base) into TMEM, this tile's sums into el / rl.
+        float el = 0.f, rl = 0.f;
+        auto exp_pass = [&](float base_used) {
+          const uint64_t nb2 = ptx::f2_pack(-base_used, -base_used);
+          uint64_t se[2];
+          float sr[4];
+#pragma unroll
+          for (int a = 0; a < 2; ++a) se[a] = ptx::f2_pack(0.f, 0.f);
+#pragma unroll
+          for (int a = 0; a < 4; ++a) sr[a] = 0.f;
+          // Four chunks of 32 keys: exponentiate, round, store each chunk.
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) {
+              const int q = ch * 16 + kk;
+              const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[2 * q], s[2 * q + 1]), c2, nb2);
+              float x0, x1, p0, p1;
+              ptx::f2_unpack(x, x0, x1);
+              if (kPolyPairPeriod > 0 &&
+                  q % (kPolyPairPeriod > 0 ? kPolyPairPeriod : 1) == kPolyPairPeriod - 1) {
+                exp2_poly_pair(x0, x1, p0, p1);
+              } else {
+                p0 = ptx::ex2_approx(x0);
+                p1 = ptx::ex2_approx(x1);
+              }
+              pk[kk] = ptx::pack_bf16x2(p0, p1);
+              se[kk & 1] = ptx::f2_add(se[kk & 1], ptx::f2_pack(p0, p1));
+              sr[(kk & 1) * 2] = ptx::add_bf16_lo(sr[(kk & 1) * 2], pk[kk]);
+              sr[(kk & 1) * 2 + 1] = ptx::add_bf16_hi(sr[(kk & 1) * 2 + 1], pk[kk]);
+            }
+            ptx::tmem_st_x16(t_s + ch * 16, pk);
+          }
+          float e0, e1;
+          ptx::f2_unpack(ptx::f2_add(se[0], se[1]), e0, e1);
+          el = e0 + e1;
+          rl = (sr[0] + sr[1]) + (sr[2] + sr[3]);
+        };
+        const float m_tile = tile_max() * c;
+        if (j == 0) {
+          m_used = m_tile;
+        } else {
+          // Rescale only rows whose maximum grew past the threshold.  TMEM
+          // access is warp-wide, so the other rows of the warp take part with
+          // a factor of exactly 1: a row's arithmetic never depends on other
+          // rows' data.
+          const bool need = m_tile > m_used + kRescaleTau;
+          if (__any_sync(0xffffffffu, need)) {
+            // O may only be touched once the previous P V product is done.
+            if (!(ok = wait_warp(bar(Lay::kOFull), (g - 1) & 1, ctl))) break;
+            ptx::tc_fence_after();
+            const float m_next = need ? m_tile : m_used;
+            const float alpha = need ? ptx::ex2_approx(m_used - m_next) : 1.f;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              ptx::tmem_ld_x32(t_o + cc * 32, o);
+#pragma unroll
+              for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+              ptx::tmem_st_x32(t_o + cc * 32, o);
+            }
+            l *= alpha;
+            l_round *= alpha;
+            m_used = m_next;
+          }
+        }
+        exp_pass(m_used == -INFINITY ? 0.f : m_used);
+        l += el;
+        l_round += rl;
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(Lay::kPFull + buf));
+      }
+      if (!ok) break;
+      // hand the row's statistics to the epilogue warps
+      if (!(ok = wait_warp(bar(Lay::kStEmpty), (st_cnt & 1) ^ 1, ctl))) break;
+      ++st_cnt;
+      stats[r] = m_used + __log2f(l);
+      stats[kBlockM + r] = 1.f / l_round;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(Lay::kStFull));
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ epilogue
+    ptx::regs_decrease<kRegsEpilogue>();
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t t_o = tmem + (static_cast<uint32_t>(wq * 32) << 16) + Lay::kTmemO;
+    uint32_t g = 0, st_cnt = 0;
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      const int u = next_unit_warp(k, ok);
+      if (u < 0) break;
+      const UnitInfo ui = decode_unit(p.work, u, H, causal);
+      if (!(ok = wait_warp(bar(Lay::kStFull), st_cnt & 1, ctl))) break;
+      ++st_cnt;
+      const float lse2 = stats[r], inv_l = stats[kBlockM + r];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(Lay::kStEmpty));
+      g += ui.n;
+      if (!(ok = wait_warp(bar(Lay::kOFull), (g - 1) & 1, ctl))) break;
+      ptx::tc_fence_after();
+      const int row_doc = ui.qb * kBlockM + r;
+      const bool row_ok = row_doc < ui.doc_len;
+      const long long token = static_cast<long long>(ui.doc_start) + row_doc;
+      uint4* orow =
+          reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + (token * H + ui.head) * D);
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        ptx::tmem_ld_x32(t_o + cc * 32, o);
+        if (cc == D / 32 - 1) {
+          // O is in registers: the tensor core may overwrite it now.
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar(Lay::kOEmpty));
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          w[q] = ptx::pack_bf16x2(__uint_as_float(o[2 * q]) * inv_l,
+                                  __uint_as_float(o[2 * q + 1]) * inv_l);
+        if (row_ok) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            orow[cc * 4 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+        }
+      }
+      if (row_ok)
+        p.lse[static_cast<long long>(ui.head) * p.total_tokens + token] =
+            lse2 * 0.69314718055994530942f;
+    }
+  } else {
+    // One setmaxnreg for the whole warpgroup (warps 8..11), as required.
+    ptx::regs_decrease<kRegsOther>();
+    if (warp == kWarpTma) {
+      // ---------------------------------------------------------- producer
+      // Lane 0 issues the copies; for MXFP8 every lane stages scale words.
+      const int n_units = p.ws_header[kWsCountOffset / 4] * H;
+      int* counter = const_cast<int*>(p.ws_header) + kWsUnitCounterOffset / 4;
+      uint32_t q_it = 0, kv_it = 0;
+      bool ok = true;
+      // One tile into the next ring slot: kind 0 = K (rows start at row0),
+      // kind 1 = V.
+      auto load_kv = [&](const UnitInfo& ui, int j, int kind) -> bool {
+        const uint32_t s = kv_it % Lay::kStages;
+        if (!wait_warp(bar(Lay::kKVEmpty + s), ((kv_it / Lay::kStages) & 1) ^ 1, ctl)) return false;
+        const uint32_t slot = sbase + Lay::kRingOff + s * Lay::kSlotBytes;
+        const int row0 = ui.doc_start + kBlockN * j;
+        if (kFp8 && kind == 0) {
+          // Scale block of the K tile: lane m0 writes keys m0 + 32 c, c = 0..3,
+          // as 16 bytes at offset 16 m0 (the layout tcgen05.cp replicates).
+          uint32_t wv[4];
+#pragma unroll
+          for (int cq = 0; cq < 4; ++cq) {
+            const int tok = row0 + lane + 32 * cq;
+            wv[cq] = tok < p.total_tokens ? p.k_scales[static_cast<long long>(tok) * H + ui.head] : 0u;
+          }
+          *reinterpret_cast<uint4*>(smem + Lay::kRingOff + s * Lay::kSlotBytes + Lay::kKBytes +
+                                    16 * lane) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (lane == 0) {
+          const int chunks = kind == 0 ? Lay::kQKChunks : Lay::kVChunks;
+          const int bytes = kind == 0 ? Lay::kKBytes : Lay::kVBytes;
+          ptx::mbar_arrive_expect_tx(bar(Lay::kKVFull + s), bytes);
+          for (int cq = 0; cq < chunks; ++cq)
+            ptx::tma_load_3d(slot + cq * Lay::kChunkBytes,
+                             kind == 0 ? static_cast<const void*>(&tm_k)
+                                       : static_cast<const void*>(&tm_v),
+                             bar(Lay::kKVFull + s), cq * (kind == 0 && kFp8 ? 128 : 64),
+                             ui.head, row0);
+        }
+        __syncwarp();
+        ++kv_it;
+        return true;
+      };
+      for (uint32_t k = 0; ok; ++k) {
+        // Claim the next unit: the first one statically, the rest from the
+        // shared counter, so each CTA takes the heaviest unit left whenever it
+        // runs out of work (the list is sorted by cost).
+        int claim = 0;
+        if (lane == 0)
+          claim = k == 0 ? static_cast<int>(blockIdx.x)
+                         : static_cast<int>(gridDim.x) + atomicAdd(counter, 1);
+        claim = __shfl_sync(0xffffffffu, claim, 0);
+        const int u = claim < n_units ? claim : -1;
+        const uint32_t uslot = k % kUnitSlots;
+        if (!(ok = wait_warp(bar(Lay::kUnitEmpty + uslot), ((k / kUnitSlots) & 1) ^ 1, ctl))) break;
+        if (lane == 0) {
+          unit_ring[uslot] = u;
+          ptx::mbar_arrive(bar(Lay::kUnitFull + uslot));
+        }
+        __syncwarp();
+        if (u < 0) break;
+        const UnitInfo ui = decode_unit(p.work, u, H, causal);
+        if (!(ok = wait_warp(bar(Lay::kQEmpty), (q_it & 1) ^ 1, ctl))) break;
+        const int qrow0 = ui.doc_start + kBlockM * ui.qb;
+        if constexpr (kFp8) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int cq = 0; cq < 4; ++cq) {
+            const int tok = qrow0 + lane + 32 * cq;
+            wv[cq] = tok < p.total_tokens ? p.q_scales[static_cast<long long>(tok) * H + ui.head] : 0u;
+          }
+          *reinterpret_cast<uint4*>(smem + Lay::kSfaOff + 16 * lane) =
+              make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(bar(Lay::kQFull), Lay::kQBytes);
+          for (int cq = 0; cq < Lay::kQKChunks; ++cq)
+            ptx::tma_load_3d(sbase + Lay::kQOff + cq * Lay::kChunkBytes, &tm_q, bar(Lay::kQFull),
+                             cq * (kFp8 ? 128 : 64), ui.head, qrow0);
+        }
+        __syncwarp();
+        ++q_it;
+        // ring order = consumption order: K_0, K_1, then V_j, K_{j+2}
+        if (!(ok = load_kv(ui, 0, 0))) break;
+        if (ui.n > 1 && !(ok = load_kv(ui, 1, 0))) break;
+        for (int j = 0; ok && j < ui.n; ++j) {
+          if (!(ok = load_kv(ui, j, 1))) break;
+          if (j + 2 < ui.n && !(ok = load_kv(ui, j + 2, 0))) break;
+        }
+      }
+      if (!ok && lane == 0) {
+        // Let copies already issued land before the CTA can exit.
+        WaitCtl drain = ctl;
+        uint32_t zero = 0;
+        drain.abort_flag = &zero;
+        const uint32_t first = kv_it > (uint32_t)Lay::kStages ? kv_it - Lay::kStages : 0;
+        for (uint32_t it = first; it < kv_it; ++it)
+          wait_one(bar(Lay::kKVFull + it % Lay::kStages), (it / Lay::kStages) & 1, drain);
+        if (q_it > 0) wait_one(bar(Lay::kQFull), (q_it - 1) & 1, drain);
+      }
+    } else if (warp == kWarpMma && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      // Descriptors are precomputed 32-bit halves (advancing along K only adds
+      // to the low half); per-buffer state is selected, never indexed.
+      constexpr uint32_t kIdescS = ptx::idesc_bf16(kBlockM, kBlockN, 0);
+      constexpr uint32_t kIdescO = ptx::idesc_bf16(kBlockM, D, 1);
+      constexpr uint32_t kDescHi = ptx::sdesc_hi_sw128(1024);
+      const uint32_t q_lo = ptx::sdesc_lo(sbase + Lay::kQOff, 16);
+      const uint32_t ring_lo = ptx::sdesc_lo(sbase + Lay::kRingOff, 16);
+      const uint32_t v_lbo = static_cast<uint32_t>(Lay::kChunkBytes - 16) >> 4 << 16;
+      uint32_t q_ph = 0, oe_cnt = 0, g = 0;
+      uint32_t cur = 0, cur_ph = 0;    // ring cursor (stage, phase)
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const uint32_t uslot = k % kUnitSlots;
+        if (!(ok = wait_one(bar(Lay::kUnitFull + uslot), (k / kUnitSlots) & 1, ctl))) break;
+        const int u = unit_ring[uslot];
+        ptx::mbar_arrive(bar(Lay::kUnitEmpty + uslot));
+        if (u < 0) break;
+        const UnitInfo ui = decode_unit(p.work, u, H, causal);
+        const int n = ui.n;
+        if (!(ok = wait_one(bar(Lay::kQFull), q_ph, ctl))) break;
+        q_ph ^= 1;
+        ptx::tc_fence_after();
+        if constexpr (kFp8)
+          tmem_cp_32x128b_x4(tmem + Lay::kTmemSfa, sf_copy_desc(sbase + Lay::kSfaOff));
+        // S for global step gs from the K tile in ring stage st
+        auto score = [&](uint32_t gs, uint32_t st) {
+          const uint32_t buf = gs & 1;
+          const uint32_t b_lo = ring_lo + st * (Lay::kSlotBytes >> 4);
+          if constexpr (kFp8) {
+            const uint32_t sfb = tmem + Lay::kTmemSfb + 4 * buf;
+            tmem_cp_32x128b_x4(sfb, sf_copy_desc(sbase + Lay::kRingOff + st * Lay::kSlotBytes +
+                                                 Lay::kKBytes));
+#pragma unroll
+            for (int kk = 0; kk < D / 32; ++kk) {
+              const uint32_t off = (kk * 32) >> 4;
+              mma_mxf8_ss(tmem + buf * 128, ptx::sdesc_join(q_lo + off, kDescHi),
+                          ptx::sdesc_join(b_lo + off, kDescHi), idesc_mxf8(kk),
+                          (static_cast<uint32_t>(kk) << 30) | (tmem + Lay::kTmemSfa),
+                          (static_cast<uint32_t>(kk) << 30) | sfb, kk > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = ((kk >> 2) * Lay::kChunkBytes + (kk & 3) * 32) >> 4;
+              ptx::mma_f16_ss(tmem + buf * 128, ptx::sdesc_join(q_lo + off, kDescHi),
+                              ptx::sdesc_join(b_lo + off, kDescHi), kIdescS, kk > 0 ? 1u : 0u);
+            }
+          }
+          ptx::mma_commit(bar(Lay::kSFull + buf));
+          ptx::mma_commit(bar(Lay::kKVEmpty + st));
+        };
+        // Next ring tile (in load order); false if the wait gave up.
+        auto take = [&](uint32_t& st) -> bool {
+          st = cur;
+          const bool r2 = wait_one(bar(Lay::kKVFull + cur), cur_ph, ctl);
+          if (++cur == static_cast<uint32_t>(Lay::kStages)) {
+            cur = 0;
+            cur_ph ^= 1;
+          }
+          return r2;
+        };
+        uint32_t st_k, st_v;
+        if (!(ok = take(st_k))) break;
+        score(g, st_k);
+        if (n > 1) {
+          if (!(ok = take(st_k))) break;
+          score(g + 1, st_k);
+        }
+        if (n <= 2) ptx::mma_commit(bar(Lay::kQEmpty));
+        for (int j = 0; j < n; ++j) {
+          const uint32_t gs = g + j;
+          const uint32_t buf = gs & 1;
+          if (!(ok = take(st_v))) break;
+          if (!(ok = wait_one(bar(Lay::kPFull + buf), (gs >> 1) & 1, ctl))) break;
+          if (j == 0 && !(ok = wait_one(bar(Lay::kOEmpty), (oe_cnt++ & 1) ^ 1, ctl))) break;
+          ptx::tc_fence_after();
+          const uint32_t b_lo = ring_lo + st_v * (Lay::kSlotBytes >> 4) + v_lbo;
+#pragma unroll
+          for (int kk = 0; kk < kBlockN / 16; ++kk)
+            ptx::mma_f16_ts(tmem + Lay::kTmemO, tmem + buf * 128 + kk * 8,
+                            ptx::sdesc_join(b_lo + kk * (2048 >> 4), kDescHi), kIdescO,
+                            (j == 0 && kk == 0) ? 0u : 1u);
+          ptx::mma_commit(bar(Lay::kOFull));
+          ptx::mma_commit(bar(Lay::kKVEmpty + st_v));
+          if (j + 2 < n) {
+            if (!(ok = take(st_k))) break;
+            score(gs + 2, st_k);
+            if (j + 2 == n - 1) ptx::mma_commit(bar(Lay::kQEmpty));
+          }
+        }
+        g += n;
+      }
+      // Every product this thread issued must be complete before TMEM is freed.
+      ptx::mma_commit(bar(Lay::kDrain));
+      WaitCtl drain = ctl;
+      uint32_t zero = 0;
+      drain.abort_flag = &zero;
+      wait_one(bar(Lay::kDrain), 0, drain);
+    }
+  }
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, Lay::kTmemCols);
+  }
+}
+
+}  // namespace attn

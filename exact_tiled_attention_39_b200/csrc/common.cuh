@@ -9,7 +9,7 @@ namespace attn {
 
 constexpr int kBlockM = 128;        // query rows per tile (one TMEM lane per row)
 constexpr int kBlockN = 128;        // keys per key/value tile
-constexpr int kTilesPerUnit = 2;    // query tiles per work unit (ping-pong pair)
+constexpr int kTilesPerUnit = 1;    // query tiles per work unit
 constexpr int kRowsPerUnit = kBlockM * kTilesPerUnit;
 
 // Workspace layout: a 256-byte header, then the work list.
@@ -25,7 +25,7 @@ constexpr size_t kWsAlign = 256;
 constexpr float kRescaleTau = 8.0f;
 
 // Upper bound of the work-list length: every document contributes
-// ceil(L / 256) <= L / 256 + 1 entries.
+// ceil(L / 128) <= L / 128 + 1 entries.
 inline int64_t max_work_entries(int64_t total_tokens, int64_t num_seqs) {
   return total_tokens / kRowsPerUnit + num_seqs + 1;
 }

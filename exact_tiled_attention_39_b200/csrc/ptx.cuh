@@ -228,6 +228,21 @@ __device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
   return d;
 }
 
+// acc + (bf16 in the low / high half of w), computed in fp32.
+__device__ __forceinline__ float add_bf16_lo(float acc, uint32_t w) {
+  float d;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tadd.rn.f32.bf16 %0, lo, %1;\n\t}"
+      : "=f"(d) : "f"(acc), "r"(w));
+  return d;
+}
+
+__device__ __forceinline__ float add_bf16_hi(float acc, uint32_t w) {
+  float d;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tadd.rn.f32.bf16 %0, hi, %1;\n\t}"
+      : "=f"(d) : "f"(acc), "r"(w));
+  return d;
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

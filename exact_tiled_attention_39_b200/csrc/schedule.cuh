@@ -8,10 +8,9 @@
 // pelatihan multi-GPU, dan kuantisasi bobot", section 1 (FlashAttention-2):
 // work is split along the sequence into query blocks.
 //
-// One entry per pair of 128-row query tiles of one document:
-// (doc_start, doc_len, pair_index, cost), cost = number of (query tile,
-// key tile) products (causal: min(qb + 1, n_kv) per query tile qb; else
-// n_kv).  Entries are sorted by cost, largest first, ties in document then
+// One entry per 128-row query tile of one document:
+// (doc_start, doc_len, query_block, cost), cost = number of key tiles it
+// needs (causal: min(qb + 1, n_kv); else n_kv).  Entries are sorted by cost, largest first, ties in document then
 // pair order, with a bitonic sort of (cost, index) keys in shared memory.
 #pragma once
 #include <cstdint>

@@ -94,9 +94,10 @@ typedef struct {
  * workspace holds the error word, the work list of the schedule-build step
  * and, for ATTN_MXFP8, the quantised operands.  Returns 0 for an invalid
  * shape.  Layout (for tests and tools): int32 error word at byte 0, int32
- * work-list length at byte 4, int32 [n][4] work list at byte 256, one entry
- * (doc_start, doc_len, pair_index, cost) per pair of 128-row query tiles,
- * sorted by cost, largest first, ties in document then pair order. */
+ * work-list length at byte 4, int32 unit counter at byte 8, int32 [n][4]
+ * work list at byte 256, one entry (doc_start, doc_len, query_block, cost)
+ * per 128-row query tile of a document, sorted by cost (key tiles needed),
+ * largest first, ties in document then query-block order. */
 size_t attn_workspace_size(const attn_shape_t* shape, attn_dtype_t dtype);
 
 /* Exact attention forward.  q, k, v: bf16 [T, H, d]; out: bf16 [T, H, d];
@@ -120,7 +121,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
  * workspace: its scratch (error word and work lists) is a 1 MiB array
  * inside the library's device image, which every GPU that loads the library
  * holds until the process exits.  Problems whose work lists need more
- * (total_tokens / 256 + num_seqs > 32751) are rejected with
+ * (total_tokens / 128 + num_seqs > 32751) are rejected with
  * ATTN_ERR_WORKSPACE before anything is launched.  Nothing is allocated: no
  * cudaMalloc, cudaFree or allocating library routine is called.
  *

@@ -10,16 +10,14 @@ loop over query blocks.  The pages fix no tile size or ordering; the reading
 taken (and implemented independently on the GPU) is:
 
   * a query tile is 128 rows of one document, counted from the document's
-    first token; a work unit is a PAIR of consecutive query tiles
-    (rows [256 t, 256 t + 256) of the document) for one head;
+    first token; a work unit is one query tile (rows [128 qb, 128 qb + 128)
+    of the document) for one head;
   * a key/value tile is 128 keys, also counted from the document start;
-  * the cost of a unit is the number of (query tile, key tile) products it
-    needs: for each query tile qb of the pair that starts inside the
-    document, min(qb + 1, n_kv) tiles when causal, n_kv otherwise, with
-    n_kv = ceil(L / 128);
+  * the cost of a unit is the number of key tiles it needs: min(qb + 1, n_kv)
+    when causal, n_kv otherwise, with n_kv = ceil(L / 128);
   * entries are sorted by cost, largest first; equal costs keep document
-    order, then pair order (a stable sort);
-  * each entry is (doc_start, doc_len, t, cost) as four int32; unit u of the
+    order, then query-block order (a stable sort);
+  * each entry is (doc_start, doc_len, qb, cost) as four int32; unit u of the
     launch is entry u // H with head u % H.
 """
 from __future__ import annotations
@@ -28,15 +26,15 @@ import numpy as np
 
 BLOCK_M = 128
 BLOCK_N = 128
-Q_TILES_PER_UNIT = 2
+Q_TILES_PER_UNIT = 1
 
 __all__ = ["schedule_ref", "unit_cost", "BLOCK_M", "BLOCK_N",
            "Q_TILES_PER_UNIT"]
 
 
 def unit_cost(L: int, t: int, causal: bool) -> int:
-    """Number of (query tile, key tile) products of pair ``t`` of a document
-    of length ``L``."""
+    """Number of key tiles needed by unit ``t`` (its query tiles) of a
+    document of length ``L``."""
     n_kv = -(-L // BLOCK_N)
     cost = 0
     for qb in range(Q_TILES_PER_UNIT * t, Q_TILES_PER_UNIT * (t + 1)):

@@ -48,7 +48,7 @@ def test_workspace_size(L):
     s = A.Shape(16384, 7, 32, 128, 4096)
     n_bf16 = A.workspace_size(s, A.ATTN_BF16)
     n_mx = A.workspace_size(s, A.ATTN_MXFP8)
-    max_entries = 16384 // 256 + 7 + 1
+    max_entries = 16384 // 128 + 7 + 1
     assert n_bf16 >= 256 + 2 * 16 * max_entries
     assert n_mx >= n_bf16 + 3 * 16384 * 32 * 128 + 3 * 16384 * 32 * 4
     assert A.workspace_size(A.Shape(16, 1, 1, 96, 16)) == 0       # d unsupported
