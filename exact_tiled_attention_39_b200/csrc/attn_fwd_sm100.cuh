@@ -20,26 +20,34 @@
 // (one per token, head and 32 head-dim elements) never span two tokens.
 //
 // A work unit is one 128-row query tile of one document and head.  On
-// sm_100a (384 threads, registers re-split per warpgroup with setmaxnreg):
+// sm_100a (512 threads, registers re-split per warpgroup with setmaxnreg):
 //
-//   warps 0..3    softmax (232 registers): one thread per query row reads its
-//                 score row from TMEM, masks, updates m and l, writes P (bf16)
-//                 back over the scores, and rescales O when its maximum grew
-//                 by more than 2^8 (lazy rescale).
-//   warps 4..7    epilogue (120 registers): O / l to bf16 and the log-sum-exp.
-//   warp 8        producer (152 registers): claims units, TMA loads of Q and of
+//   warps 0..7    softmax (168 registers), two warpgroups on the same rows:
+//                 warpgroup h takes keys [64 h, 64 h + 64) of every score
+//                 tile.  Each thread reads its half row from TMEM and masks
+//                 it; the two halves swap their maxima through shared memory,
+//                 so both use the same running maximum m; each writes its
+//                 half of P (bf16) back over its own scores, keeps its part of
+//                 l, and rescales its half of O when the row maximum grew by
+//                 more than 2^8 (lazy rescale).
+//   warps 8..11   epilogue (96 registers): O / l to bf16 and the log-sum-exp.
+//   warp 12       producer (80 registers): claims units, TMA loads of Q and of
 //                 K_j, V_j into a ring of shared-memory slots; for MXFP8 the
 //                 whole warp also stages the E8M0 scale blocks.
-//   warp 9        MMA issuer (one thread): S = Q K_j^T into one of two TMEM
+//   warp 13       MMA issuer (one thread): S = Q K_j^T into one of two TMEM
 //                 score buffers, O += P V_j with P read from TMEM.
-//   warps 10..11  idle.
+//   warps 14..15  idle.
 //
 // The score buffers alternate between key steps, so while the softmax works
-// on step j the tensor core computes P_{j-1} V_{j-1} and S_{j+1}.
+// on step j the tensor core computes P_{j-1} V_{j-1} and S_{j+1}.  Splitting
+// a row between two warps halves the softmax latency of a step and puts two
+// softmax warps on every SM sub-partition, which keeps the exponential unit
+// fed while the other warp waits on a dependency.
 //
-// TMEM (512 columns, lane = query row): S buffers at columns 0 and 128 (P
-// overwrites the first 64 columns of its buffer), O at 256; for MXFP8 the
-// scale factors of Q at 384 and of the current K tile at 388 / 392.
+// TMEM (512 columns, lane = query row): S buffers at columns 0 and 128 (the
+// P half of warpgroup h overwrites columns [64 h, 64 h + 32) of its buffer),
+// O at 256; for MXFP8 the scale factors of Q at 384 and of the current K tile
+// at 388 / 392.
 #pragma once
 #include <cuda.h>
 
@@ -65,18 +73,20 @@ struct FwdParams {
   unsigned long long timeout_ns;
 };
 
-constexpr int kFwdThreads = 384;
-// Registers per thread at launch: 65536 / 384 rounded down to a multiple of 8.
-// Each warpgroup moves once, at the start of its role, and keeps that count:
-// a warpgroup that lowered its count and raised it again could take back
-// registers before the softmax warpgroup's increase is served.
-constexpr uint32_t kRegsEntry = 168;
-constexpr uint32_t kRegsSoftmax = 232, kRegsEpilogue = 120, kRegsOther = 152;
-static_assert(kRegsSoftmax + kRegsEpilogue + kRegsOther == 3 * kRegsEntry,
+constexpr int kFwdThreads = 512;
+// Registers per thread at launch: 65536 / 512.  Each warpgroup moves once, at
+// the start of its role, and keeps that count: a warpgroup that lowered its
+// count and raised it again could take back registers before the softmax
+// warpgroups' increase is served.
+constexpr uint32_t kRegsEntry = 128;
+constexpr uint32_t kRegsSoftmax = 168, kRegsEpilogue = 96, kRegsOther = 80;
+static_assert(2 * kRegsSoftmax + kRegsEpilogue + kRegsOther == 4 * kRegsEntry,
               "register split must use exactly the registers the CTA is launched with");
 
+constexpr int kSoftmaxWarps = 8;            // two warpgroups, one per half of the keys
+constexpr int kHalfKeys = kBlockN / 2;
 constexpr int kUnitSlots = 4;
-constexpr int kUnitConsumers = 1 + 4 + 4;   // MMA thread + softmax warps + epilogue warps
+constexpr int kUnitConsumers = 1 + kSoftmaxWarps + 4;   // MMA thread + softmax + epilogue warps
 
 // Exponentials: most run on the MUFU unit (ex2.approx); pairs of keys with
 // index k % period == period - 1 run on the FMA pipe instead, as 2^x =
@@ -110,11 +120,14 @@ struct FwdLayout {
   static constexpr int kQOff = 0;
   static constexpr int kSfaOff = kQBytes;                     // MXFP8 only
   static constexpr int kRingOff = ((kQBytes + (kFp8 ? kSfBytes : 0)) + 1023) / 1024 * 1024;
-  static constexpr int kReserve = 4096;                       // stats, barriers, ring of units
+  static constexpr int kReserve = 6144;                       // stats, maxima, barriers, units
   static constexpr int kStagesFit = (232448 - kRingOff - kReserve) / kSlotBytes;
   static constexpr int kStages = kStagesFit > 10 ? 10 : kStagesFit;
-  static constexpr int kStatsOff = kRingOff + kStages * kSlotBytes;   // float [2][128]
-  static constexpr int kBarOff = kStatsOff + 2 * kBlockM * 4;
+  // Unit statistics handed to the epilogue: float [5][128] = m, then l and
+  // the rounded l of each half.  Half-row maxima: float [2 steps][2][128].
+  static constexpr int kStatsOff = kRingOff + kStages * kSlotBytes;
+  static constexpr int kXmaxOff = kStatsOff + 5 * kBlockM * 4;
+  static constexpr int kBarOff = kXmaxOff + 2 * 2 * kBlockM * 4;
   static constexpr int kQFull = 0, kQEmpty = 1;
   static constexpr int kKVFull = 2;                           // + stage
   static constexpr int kKVEmpty = kKVFull + kStages;          // + stage
@@ -124,7 +137,8 @@ struct FwdLayout {
   static constexpr int kOEmpty = kOFull + 1;
   static constexpr int kStFull = kOEmpty + 1;
   static constexpr int kStEmpty = kStFull + 1;
-  static constexpr int kDrain = kStEmpty + 1;
+  static constexpr int kXFull = kStEmpty + 1;                // + step parity
+  static constexpr int kDrain = kXFull + 2;
   static constexpr int kUnitFull = kDrain + 1;                // + slot
   static constexpr int kUnitEmpty = kUnitFull + kUnitSlots;   // + slot
   static constexpr int kNumBars = kUnitEmpty + kUnitSlots;
@@ -284,10 +298,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   auto bar = [&](int i) -> uint32_t { return sbase + Lay::kBarOff + 8 * i; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile uint32_t* abort_flag = tmem_holder + 1;
-  float* stats = reinterpret_cast<float*>(smem + Lay::kStatsOff);   // [lse2, 1/l_round][row]
+  float* stats = reinterpret_cast<float*>(smem + Lay::kStatsOff);   // [m, l0, lr0, l1, lr1][row]
+  float* xmax = reinterpret_cast<float*>(smem + Lay::kXmaxOff);     // [step & 1][half][row]
   volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + Lay::kUnitOff);
 
-  constexpr int kWarpTma = 8, kWarpMma = 9;
+  constexpr int kWarpTma = 12, kWarpMma = 13;
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(Lay::kQFull), 1);
     ptx::mbar_init(bar(Lay::kQEmpty), 1);
@@ -297,11 +312,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(bar(Lay::kSFull + b), 1);
-      ptx::mbar_init(bar(Lay::kPFull + b), 4);    // one arrival per softmax warp
+      ptx::mbar_init(bar(Lay::kPFull + b), kSoftmaxWarps);   // one arrival per softmax warp
+      ptx::mbar_init(bar(Lay::kXFull + b), kSoftmaxWarps);
     }
     ptx::mbar_init(bar(Lay::kOFull), 1);
     ptx::mbar_init(bar(Lay::kOEmpty), 4);         // one arrival per epilogue warp
-    ptx::mbar_init(bar(Lay::kStFull), 4);
+    ptx::mbar_init(bar(Lay::kStFull), kSoftmaxWarps);
     ptx::mbar_init(bar(Lay::kStEmpty), 4);
     ptx::mbar_init(bar(Lay::kDrain), 1);
     for (int i = 0; i < kUnitSlots; ++i) {
@@ -343,12 +359,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     return u;
   };
 
-  if (warp < 4) {
+  if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax
     ptx::regs_increase<kRegsSoftmax>();
-    const int r = warp * 32 + lane;               // query row within the tile
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t t_o = tmem + lane_off + Lay::kTmemO;
+    const int h = warp >> 2;                      // which half of the keys
+    const int r = (warp & 3) * 32 + lane;         // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t t_o = tmem + lane_off + Lay::kTmemO + h * (D / 2);
     const float c = p.scale_log2;
     const uint64_t c2 = ptx::f2_pack(c, c);
     uint32_t g = 0, st_cnt = 0;                   // global key step, units handed over
@@ -357,61 +374,89 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int u = next_unit_warp(k, ok);
       if (u < 0) break;
       const UnitInfo ui = decode_unit(p.work, u, H, causal);
-      float m_used = -INFINITY;   // running maximum in log2 units
-      float l = 0.f;              // sum of the weights
-      float l_round = 0.f;        // sum of the weights as rounded to bf16
+      float m_used = -INFINITY;   // running maximum in log2 units (same in both halves)
+      float l = 0.f;              // this half's sum of the weights
+      float l_round = 0.f;        // the same, of the weights as rounded to bf16
       for (int j = 0; j < ui.n; ++j, ++g) {
         const uint32_t buf = g & 1;
-        const uint32_t t_s = tmem + lane_off + buf * 128;
+        const uint32_t t_s = tmem + lane_off + buf * 128 + h * kHalfKeys;
         if (!(ok = wait_warp(bar(Lay::kSFull + buf), (g >> 1) & 1, ctl))) break;
         ptx::tc_fence_after();
-        uint32_t sa[64], sb[64];
+        uint32_t sa[64];
         ptx::tmem_ld_x64(t_s, sa);
-        ptx::tmem_ld_x64(t_s + 64, sb);
-        float s[128];
+        float s[64];
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
-          s[q] = __uint_as_float(sa[q]);
-          s[64 + q] = __uint_as_float(sb[q]);
-        }
+        for (int q = 0; q < 64; ++q) s[q] = __uint_as_float(sa[q]);
         const bool diag = causal && j == ui.qb;
         if (diag || (j + 1) * kBlockN > ui.doc_len) {
           int limit = ui.doc_len - j * kBlockN;
           if (diag) limit = min(limit, r + 1);
+          limit -= h * kHalfKeys;
 #pragma unroll
-          for (int q = 0; q < 128; ++q)
+          for (int q = 0; q < 64; ++q)
             if (q >= limit) s[q] = -INFINITY;
         }
-        // Row maximum of the tile (8 independent chains).
-        auto tile_max = [&]() -> float {
-          float mx[8];
+        // Maximum of this half (8 independent chains), then of the row: the
+        // two halves swap theirs through shared memory.
+        float mx[8];
 #pragma unroll
-          for (int a = 0; a < 8; ++a) mx[a] = fmaxf(s[2 * a], s[2 * a + 1]);
+        for (int a = 0; a < 8; ++a) mx[a] = fmaxf(s[2 * a], s[2 * a + 1]);
 #pragma unroll
-          for (int q = 16; q < 128; q += 16)
+        for (int q = 16; q < 64; q += 16)
 #pragma unroll
-            for (int a = 0; a < 8; ++a) mx[a] = ptx::fmax3(mx[a], s[q + 2 * a], s[q + 2 * a + 1]);
-          return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        };
+          for (int a = 0; a < 8; ++a) mx[a] = ptx::fmax3(mx[a], s[q + 2 * a], s[q + 2 * a + 1]);
+        const float m_half = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        float* xm = xmax + buf * 2 * kBlockM;
+        xm[h * kBlockM + r] = m_half;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(Lay::kXFull + buf));
+        if (!(ok = wait_warp(bar(Lay::kXFull + buf), (g >> 1) & 1, ctl))) break;
+        const float m_tile = fmaxf(m_half, xm[(h ^ 1) * kBlockM + r]) * c;
+        if (j == 0) {
+          m_used = m_tile;
+        } else {
+          // Rescale only rows whose maximum grew past the threshold.  TMEM
+          // access is warp-wide, so the other rows of the warp take part with
+          // a factor of exactly 1: a row's arithmetic never depends on other
+          // rows' data.  Both halves of a row take the same decision.
+          const bool need = m_tile > m_used + kRescaleTau;
+          if (__any_sync(0xffffffffu, need)) {
+            // O may only be touched once the previous P V product is done.
+            if (!(ok = wait_warp(bar(Lay::kOFull), (g - 1) & 1, ctl))) break;
+            ptx::tc_fence_after();
+            const float m_next = need ? m_tile : m_used;
+            const float alpha = need ? ptx::ex2_approx(m_used - m_next) : 1.f;
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc) {
+              uint32_t o[32];
+              ptx::tmem_ld_x32(t_o + cc * 32, o);
+#pragma unroll
+              for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+              ptx::tmem_st_x32(t_o + cc * 32, o);
+            }
+            l *= alpha;
+            l_round *= alpha;
+            m_used = m_next;
+          }
+        }
         // Weights are rounded to bf16 for the P V product.  Two normalisers:
         // l_round sums the rounded weights, so O / l_round is an exact convex
         // combination of the values with the weights actually used (no bias
         // from the rounding, which matters when one key dominates a row);
         // l sums the unrounded weights and gives the log-sum-exp.
-        // exp_pass: P = 2^(s c - base) into TMEM, this tile's sums into el / rl.
-        float el = 0.f, rl = 0.f;
-        auto exp_pass = [&](float base_used) {
-          const uint64_t nb2 = ptx::f2_pack(-base_used, -base_used);
+        {
+          const float base = m_used == -INFINITY ? 0.f : m_used;
+          const uint64_t nb2 = ptx::f2_pack(-base, -base);
           uint64_t se[2];
           float sr[4];
 #pragma unroll
           for (int a = 0; a < 2; ++a) se[a] = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
           for (int a = 0; a < 4; ++a) sr[a] = 0.f;
-          // Four chunks of 32 keys: exponentiate, round, store each chunk.
+          // Two chunks of 32 keys: exponentiate, round, store each chunk.
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
+          for (int ch = 0; ch < 2; ++ch) {
             uint32_t pk[16];
 #pragma unroll
             for (int kk = 0; kk < 16; ++kk) {
@@ -435,40 +480,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           float e0, e1;
           ptx::f2_unpack(ptx::f2_add(se[0], se[1]), e0, e1);
-          el = e0 + e1;
-          rl = (sr[0] + sr[1]) + (sr[2] + sr[3]);
-        };
-        const float m_tile = tile_max() * c;
-        if (j == 0) {
-          m_used = m_tile;
-        } else {
-          // Rescale only rows whose maximum grew past the threshold.  TMEM
-          // access is warp-wide, so the other rows of the warp take part with
-          // a factor of exactly 1: a row's arithmetic never depends on other
-          // rows' data.
-          const bool need = m_tile > m_used + kRescaleTau;
-          if (__any_sync(0xffffffffu, need)) {
-            // O may only be touched once the previous P V product is done.
-            if (!(ok = wait_warp(bar(Lay::kOFull), (g - 1) & 1, ctl))) break;
-            ptx::tc_fence_after();
-            const float m_next = need ? m_tile : m_used;
-            const float alpha = need ? ptx::ex2_approx(m_used - m_next) : 1.f;
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-              uint32_t o[32];
-              ptx::tmem_ld_x32(t_o + cc * 32, o);
-#pragma unroll
-              for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-              ptx::tmem_st_x32(t_o + cc * 32, o);
-            }
-            l *= alpha;
-            l_round *= alpha;
-            m_used = m_next;
-          }
+          l += e0 + e1;
+          l_round += (sr[0] + sr[1]) + (sr[2] + sr[3]);
         }
-        exp_pass(m_used == -INFINITY ? 0.f : m_used);
-        l += el;
-        l_round += rl;
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
@@ -478,12 +492,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // hand the row's statistics to the epilogue warps
       if (!(ok = wait_warp(bar(Lay::kStEmpty), (st_cnt & 1) ^ 1, ctl))) break;
       ++st_cnt;
-      stats[r] = m_used + __log2f(l);
-      stats[kBlockM + r] = 1.f / l_round;
+      if (h == 0) stats[r] = m_used;
+      stats[(1 + 2 * h) * kBlockM + r] = l;
+      stats[(2 + 2 * h) * kBlockM + r] = l_round;
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(Lay::kStFull));
     }
-  } else if (warp < 8) {
+  } else if (warp < kSoftmaxWarps + 4) {
     // ------------------------------------------------------------ epilogue
     ptx::regs_decrease<kRegsEpilogue>();
     const int wq = warp & 3;
@@ -497,7 +512,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const UnitInfo ui = decode_unit(p.work, u, H, causal);
       if (!(ok = wait_warp(bar(Lay::kStFull), st_cnt & 1, ctl))) break;
       ++st_cnt;
-      const float lse2 = stats[r], inv_l = stats[kBlockM + r];
+      const float lse2 = stats[r] + __log2f(stats[kBlockM + r] + stats[3 * kBlockM + r]);
+      const float inv_l = 1.f / (stats[2 * kBlockM + r] + stats[4 * kBlockM + r]);
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(Lay::kStEmpty));
       g += ui.n;
@@ -534,7 +550,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             lse2 * 0.69314718055994530942f;
     }
   } else {
-    // One setmaxnreg for the whole warpgroup (warps 8..11), as required.
+    // One setmaxnreg for the whole warpgroup (warps 12..15), as required.
     ptx::regs_decrease<kRegsOther>();
     if (warp == kWarpTma) {
       // ---------------------------------------------------------- producer
@@ -719,7 +735,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const uint32_t b_lo = ring_lo + st_v * (Lay::kSlotBytes >> 4) + v_lbo;
 #pragma unroll
           for (int kk = 0; kk < kBlockN / 16; ++kk)
-            ptx::mma_f16_ts(tmem + Lay::kTmemO, tmem + buf * 128 + kk * 8,
+            ptx::mma_f16_ts(tmem + Lay::kTmemO,
+                            tmem + buf * 128 + (kk >> 2) * kHalfKeys + (kk & 3) * 8,
                             ptx::sdesc_join(b_lo + kk * (2048 >> 4), kDescHi), kIdescO,
                             (j == 0 && kk == 0) ? 0u : 1u);
           ptx::mma_commit(bar(Lay::kOFull));
