@@ -224,15 +224,24 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   const bool fp8_kernel = dtype == ATTN_MXFP8 && s.head_dim == 128;
   const void* qk_src[2] = {q, k};
   if (dtype == ATTN_MXFP8) {
+    // One launch for all three tensors.  The block-scaled kernel reads the
+    // codes and scales of Q and K and the exact dequantised V; the head-dim
+    // 64 fallback reads dequantised Q, K and V.
     const void* src[3] = {q, k, v};
     const long long n_blocks =
         static_cast<long long>(s.total_tokens) * s.num_heads * (s.head_dim / 32);
-    const unsigned qgrid = static_cast<unsigned>((n_blocks + 255) / 256);
+    QuantJobs jobs;
+    jobs.n_blocks = n_blocks;
     for (int i = 0; i < 3; ++i) {
-      quantize_mxfp8_kernel<<<qgrid, 256, 0, strm>>>(
-          static_cast<const uint4*>(src[i]), reinterpret_cast<uint4*>(ws + wl.codes_off[i]),
-          ws + wl.scales_off[i], reinterpret_cast<uint4*>(ws + wl.deq_off[i]), n_blocks);
+      const bool use_codes = fp8_kernel && i < 2;
+      jobs.t[i].x = static_cast<const uint4*>(src[i]);
+      jobs.t[i].codes = use_codes ? reinterpret_cast<uint4*>(ws + wl.codes_off[i]) : nullptr;
+      jobs.t[i].scales = use_codes ? ws + wl.scales_off[i] : nullptr;
+      jobs.t[i].deq = use_codes ? nullptr : reinterpret_cast<uint4*>(ws + wl.deq_off[i]);
     }
+    const long long qgrid = (n_blocks + 255) / 256;
+    if (qgrid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    quantize_mxfp8_qkv_kernel<<<dim3(static_cast<unsigned>(qgrid), 3), 256, 0, strm>>>(jobs);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     for (int i = 0; i < 2; ++i) qk_src[i] = ws + (fp8_kernel ? wl.codes_off[i] : wl.deq_off[i]);
     v = ws + wl.deq_off[2];

@@ -98,6 +98,17 @@ constexpr int kUnitConsumers = 1 + kSoftmaxWarps + 4;   // MMA thread + softmax 
 #endif
 constexpr int kPolyPairPeriod = ATTN_POLY_PAIR_PERIOD;
 
+// Separate-P path: each softmax half reads the other half's scores from TMEM
+// for the row maximum instead of swapping maxima through shared memory.
+#ifndef ATTN_MAX_FROM_TMEM
+#define ATTN_MAX_FROM_TMEM 0
+#endif
+// bf16: P in buffers of its own (1) or over the scores (0).
+#ifndef ATTN_SEPARATE_P
+#define ATTN_SEPARATE_P 1
+#endif
+constexpr bool kMaxFromTmem = ATTN_MAX_FROM_TMEM != 0;
+
 // 2^f on [0, 1): 1 + f (c1 + f (c2 + f c3)), a minimax fit of the relative
 // error (max 8.6e-5) made by csrc/fit_exp2_poly.py; p(0) = 1 exactly.
 constexpr float kExp2C1 = 6.951168180e-01f;
@@ -133,22 +144,32 @@ struct FwdLayout {
   static constexpr int kKVEmpty = kKVFull + kStages;          // + stage
   static constexpr int kSFull = kKVEmpty + kStages;           // + buffer
   static constexpr int kPFull = kSFull + 2;                   // + buffer
-  static constexpr int kOFull = kPFull + 2;
-  static constexpr int kOEmpty = kOFull + 1;
+  // O of a unit complete (one phase per unit: a waiter is never more than one
+  // phase behind, which a parity wait needs)
+  static constexpr int kOUnit = kPFull + 2;
+  static constexpr int kOEmpty = kOUnit + 1;
   static constexpr int kStFull = kOEmpty + 1;
   static constexpr int kStEmpty = kStFull + 1;
   static constexpr int kXFull = kStEmpty + 1;                // + step parity
-  static constexpr int kDrain = kXFull + 2;
+  static constexpr int kSFree = kXFull + 2;                   // + buffer (bf16 only)
+  static constexpr int kPFree = kSFree + 2;                   // + buffer: P V of that buffer done
+  static constexpr int kDrain = kPFree + 2;
   static constexpr int kUnitFull = kDrain + 1;                // + slot
   static constexpr int kUnitEmpty = kUnitFull + kUnitSlots;   // + slot
   static constexpr int kNumBars = kUnitEmpty + kUnitSlots;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;     // tmem base, abort flag
-  static constexpr int kUnitOff = kMiscOff + 16;              // int32 [kUnitSlots]
-  static constexpr int kBytes = kUnitOff + 4 * kUnitSlots;
+  static constexpr int kMiscOff = (kBarOff + kNumBars * 8 + 15) / 16 * 16;   // tmem base, abort flag
+  static constexpr int kUnitOff = kMiscOff + 16;              // int4 [kUnitSlots]
+  static constexpr int kBytes = kUnitOff + 16 * kUnitSlots;
   static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
   static_assert(kBytes - kStatsOff <= kReserve, "reserve too small");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemO = 256, kTmemSfa = 384, kTmemSfb = 388;
+  // bf16: P has buffers of its own (64 columns each) after O, so the next
+  // score product can overwrite a score buffer as soon as the softmax has
+  // read it.  MXFP8 needs those columns for the scale factors and writes P
+  // over the scores instead.
+  static constexpr bool kSepP = !kFp8 && ATTN_SEPARATE_P != 0;
+  static constexpr uint32_t kTmemP = 384;
 };
 
 // Bounded waits.  A wait gives up when the CTA's abort flag is raised or
@@ -205,13 +226,13 @@ struct UnitInfo {
   int doc_start, doc_len, qb, head, kv_tiles, n;   // n = key steps of this tile
 };
 
-__device__ __forceinline__ UnitInfo decode_unit(const int4* work, int u, int H, int causal) {
-  const int4 w = work[u / H];
+// Unit from its ring entry (doc_start, doc_len, query block, head).
+__device__ __forceinline__ UnitInfo decode_unit(int4 w, int causal) {
   UnitInfo r;
   r.doc_start = w.x;
   r.doc_len = w.y;
   r.qb = w.z;
-  r.head = u % H;
+  r.head = w.w;
   r.kv_tiles = (w.y + kBlockN - 1) / kBlockN;
   r.n = causal ? min(w.z + 1, r.kv_tiles) : r.kv_tiles;
   return r;
@@ -300,7 +321,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   volatile uint32_t* abort_flag = tmem_holder + 1;
   float* stats = reinterpret_cast<float*>(smem + Lay::kStatsOff);   // [m, l0, lr0, l1, lr1][row]
   float* xmax = reinterpret_cast<float*>(smem + Lay::kXmaxOff);     // [step & 1][half][row]
-  volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + Lay::kUnitOff);
+  // Units handed from the producer to the other roles, decoded (doc_len < 0
+  // marks the end of the work).
+  int4* unit_ring = reinterpret_cast<int4*>(smem + Lay::kUnitOff);
 
   constexpr int kWarpTma = 12, kWarpMma = 13;
   if (threadIdx.x == 0) {
@@ -314,8 +337,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ptx::mbar_init(bar(Lay::kSFull + b), 1);
       ptx::mbar_init(bar(Lay::kPFull + b), kSoftmaxWarps);   // one arrival per softmax warp
       ptx::mbar_init(bar(Lay::kXFull + b), kSoftmaxWarps);
+      ptx::mbar_init(bar(Lay::kSFree + b), kSoftmaxWarps);
+      ptx::mbar_init(bar(Lay::kPFree + b), 1);
     }
-    ptx::mbar_init(bar(Lay::kOFull), 1);
+    ptx::mbar_init(bar(Lay::kOUnit), 1);
     ptx::mbar_init(bar(Lay::kOEmpty), 4);         // one arrival per epilogue warp
     ptx::mbar_init(bar(Lay::kStFull), kSoftmaxWarps);
     ptx::mbar_init(bar(Lay::kStEmpty), 4);
@@ -348,15 +373,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const WaitCtl ctl{abort_flag, p.err, p.timeout_ns};
   const int H = p.num_heads;
   const int causal = p.causal;
-  // Consumer side of the unit ring: the k-th unit of this CTA, or -1 when the
-  // work is exhausted (also -1 if the wait gave up; `ok` says which).
-  auto next_unit_warp = [&](uint32_t k, bool& ok) -> int {
+  // Consumer side of the unit ring: the k-th unit of this CTA; doc_len < 0
+  // when the work is exhausted (also if the wait gave up; `ok` says which).
+  auto next_unit_warp = [&](uint32_t k, bool& ok) -> int4 {
     const uint32_t slot = k % kUnitSlots;
-    if (!(ok = wait_warp(bar(Lay::kUnitFull + slot), (k / kUnitSlots) & 1, ctl))) return -1;
-    const int u = unit_ring[slot];
+    if (!(ok = wait_warp(bar(Lay::kUnitFull + slot), (k / kUnitSlots) & 1, ctl)))
+      return make_int4(0, -1, 0, 0);
+    const int4 w = unit_ring[slot];   // after the wait (asm with a memory clobber)
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(bar(Lay::kUnitEmpty + slot));
-    return u;
+    return w;
   };
 
   if (warp < kSoftmaxWarps) {
@@ -371,9 +397,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint32_t g = 0, st_cnt = 0;                   // global key step, units handed over
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
-      const int u = next_unit_warp(k, ok);
-      if (u < 0) break;
-      const UnitInfo ui = decode_unit(p.work, u, H, causal);
+      const int4 uw = next_unit_warp(k, ok);
+      if (uw.y < 0) break;
+      const UnitInfo ui = decode_unit(uw, causal);
       float m_used = -INFINITY;   // running maximum in log2 units (same in both halves)
       float l = 0.f;              // this half's sum of the weights
       float l_round = 0.f;        // the same, of the weights as rounded to bf16
@@ -407,12 +433,46 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int a = 0; a < 8; ++a) mx[a] = ptx::fmax3(mx[a], s[q + 2 * a], s[q + 2 * a + 1]);
         const float m_half = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        float* xm = xmax + buf * 2 * kBlockM;
-        xm[h * kBlockM + r] = m_half;
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(Lay::kXFull + buf));
-        if (!(ok = wait_warp(bar(Lay::kXFull + buf), (g >> 1) & 1, ctl))) break;
-        const float m_tile = fmaxf(m_half, xm[(h ^ 1) * kBlockM + r]) * c;
+        float m_other;
+        if constexpr (Lay::kSepP && kMaxFromTmem) {
+          // The other half's scores stay in TMEM until both halves have read
+          // them (P has buffers of its own), so its maximum is read there.
+          const uint32_t t_x = tmem + lane_off + buf * 128 + (h ^ 1) * kHalfKeys;
+          int limit_x = kHalfKeys;
+          if (diag || (j + 1) * kBlockN > ui.doc_len) {
+            limit_x = ui.doc_len - j * kBlockN;
+            if (diag) limit_x = min(limit_x, r + 1);
+            limit_x -= (h ^ 1) * kHalfKeys;
+          }
+          float mo[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t xo[32];
+            ptx::tmem_ld_x32(t_x + cc * 32, xo);
+#pragma unroll
+            for (int q = 0; q < 32; q += 2) {
+              const int kq = cc * 32 + q;
+              const float a0 = kq < limit_x ? __uint_as_float(xo[q]) : -INFINITY;
+              const float a1 = kq + 1 < limit_x ? __uint_as_float(xo[q + 1]) : -INFINITY;
+              mo[(q >> 1) & 3] = ptx::fmax3(mo[(q >> 1) & 3], a0, a1);
+            }
+          }
+          m_other = fmaxf(fmaxf(mo[0], mo[1]), fmaxf(mo[2], mo[3]));
+        } else {
+          float* xm = xmax + buf * 2 * kBlockM;
+          xm[h * kBlockM + r] = m_half;
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar(Lay::kXFull + buf));
+          if (!(ok = wait_warp(bar(Lay::kXFull + buf), (g >> 1) & 1, ctl))) break;
+          m_other = xm[(h ^ 1) * kBlockM + r];
+        }
+        if constexpr (Lay::kSepP) {
+          // both halves' scores are in registers: the buffer may take S_{j+2}
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar(Lay::kSFree + buf));
+        }
+        const float m_tile = fmaxf(m_half, m_other) * c;
         if (j == 0) {
           m_used = m_tile;
         } else {
@@ -423,7 +483,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const bool need = m_tile > m_used + kRescaleTau;
           if (__any_sync(0xffffffffu, need)) {
             // O may only be touched once the previous P V product is done.
-            if (!(ok = wait_warp(bar(Lay::kOFull), (g - 1) & 1, ctl))) break;
+            // Its buffer's barrier has one phase per two steps and this warp
+            // has seen the phase before (P V two steps further back) complete
+            // already, so the parity names exactly P_{j-1} V_{j-1}.
+            if (!(ok = wait_warp(bar(Lay::kPFree + ((g - 1) & 1)), ((g - 1) >> 1) & 1, ctl))) break;
             ptx::tc_fence_after();
             const float m_next = need ? m_tile : m_used;
             const float alpha = need ? ptx::ex2_approx(m_used - m_next) : 1.f;
@@ -445,6 +508,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // combination of the values with the weights actually used (no bias
         // from the rounding, which matters when one key dominates a row);
         // l sums the unrounded weights and gives the log-sum-exp.
+        // P of this step goes to its own buffer (bf16) once the P V product
+        // two steps back has read it, else over this half's scores (which
+        // that product has read as well: this step's scores came after it).
+        // The wait is taken on both paths, after the weights are formed; it
+        // also keeps this warp at most one phase behind each buffer's barrier.
+        const uint32_t t_p =
+            Lay::kSepP ? tmem + lane_off + Lay::kTmemP + buf * (kBlockN / 2) + h * (kHalfKeys / 2)
+                       : t_s;
         {
           const float base = m_used == -INFINITY ? 0.f : m_used;
           const uint64_t nb2 = ptx::f2_pack(-base, -base);
@@ -454,34 +525,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int a = 0; a < 2; ++a) se[a] = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
           for (int a = 0; a < 4; ++a) sr[a] = 0.f;
-          // Two chunks of 32 keys: exponentiate, round, store each chunk.
+          uint32_t pk[32];
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk) {
-              const int q = ch * 16 + kk;
-              const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[2 * q], s[2 * q + 1]), c2, nb2);
-              float x0, x1, p0, p1;
-              ptx::f2_unpack(x, x0, x1);
-              if (kPolyPairPeriod > 0 &&
-                  q % (kPolyPairPeriod > 0 ? kPolyPairPeriod : 1) == kPolyPairPeriod - 1) {
-                exp2_poly_pair(x0, x1, p0, p1);
-              } else {
-                p0 = ptx::ex2_approx(x0);
-                p1 = ptx::ex2_approx(x1);
-              }
-              pk[kk] = ptx::pack_bf16x2(p0, p1);
-              se[kk & 1] = ptx::f2_add(se[kk & 1], ptx::f2_pack(p0, p1));
-              sr[(kk & 1) * 2] = ptx::add_bf16_lo(sr[(kk & 1) * 2], pk[kk]);
-              sr[(kk & 1) * 2 + 1] = ptx::add_bf16_hi(sr[(kk & 1) * 2 + 1], pk[kk]);
+          for (int q = 0; q < 32; ++q) {
+            const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[2 * q], s[2 * q + 1]), c2, nb2);
+            float x0, x1, p0, p1;
+            ptx::f2_unpack(x, x0, x1);
+            if (kPolyPairPeriod > 0 &&
+                q % (kPolyPairPeriod > 0 ? kPolyPairPeriod : 1) == kPolyPairPeriod - 1) {
+              exp2_poly_pair(x0, x1, p0, p1);
+            } else {
+              p0 = ptx::ex2_approx(x0);
+              p1 = ptx::ex2_approx(x1);
             }
-            ptx::tmem_st_x16(t_s + ch * 16, pk);
+            pk[q] = ptx::pack_bf16x2(p0, p1);
+            se[q & 1] = ptx::f2_add(se[q & 1], ptx::f2_pack(p0, p1));
+            sr[(q & 1) * 2] = ptx::add_bf16_lo(sr[(q & 1) * 2], pk[q]);
+            sr[(q & 1) * 2 + 1] = ptx::add_bf16_hi(sr[(q & 1) * 2 + 1], pk[q]);
           }
           float e0, e1;
           ptx::f2_unpack(ptx::f2_add(se[0], se[1]), e0, e1);
           l += e0 + e1;
           l_round += (sr[0] + sr[1]) + (sr[2] + sr[3]);
+          if (!(ok = wait_warp(bar(Lay::kPFree + buf), ((g >> 1) & 1) ^ 1, ctl))) break;
+          ptx::tc_fence_after();
+          ptx::tmem_st_x32(t_p, pk);
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
@@ -504,20 +572,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t t_o = tmem + (static_cast<uint32_t>(wq * 32) << 16) + Lay::kTmemO;
-    uint32_t g = 0, st_cnt = 0;
+    uint32_t st_cnt = 0;
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
-      const int u = next_unit_warp(k, ok);
-      if (u < 0) break;
-      const UnitInfo ui = decode_unit(p.work, u, H, causal);
+      const int4 uw = next_unit_warp(k, ok);
+      if (uw.y < 0) break;
+      const UnitInfo ui = decode_unit(uw, causal);
       if (!(ok = wait_warp(bar(Lay::kStFull), st_cnt & 1, ctl))) break;
       ++st_cnt;
       const float lse2 = stats[r] + __log2f(stats[kBlockM + r] + stats[3 * kBlockM + r]);
       const float inv_l = 1.f / (stats[2 * kBlockM + r] + stats[4 * kBlockM + r]);
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(Lay::kStEmpty));
-      g += ui.n;
-      if (!(ok = wait_warp(bar(Lay::kOFull), (g - 1) & 1, ctl))) break;
+      if (!(ok = wait_warp(bar(Lay::kOUnit), k & 1, ctl))) break;
       ptx::tc_fence_after();
       const int row_doc = ui.qb * kBlockM + r;
       const bool row_ok = row_doc < ui.doc_len;
@@ -604,16 +671,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           claim = k == 0 ? static_cast<int>(blockIdx.x)
                          : static_cast<int>(gridDim.x) + atomicAdd(counter, 1);
         claim = __shfl_sync(0xffffffffu, claim, 0);
-        const int u = claim < n_units ? claim : -1;
+        int4 uw = make_int4(0, -1, 0, 0);
+        if (claim < n_units) {
+          const int4 e = p.work[claim / H];
+          uw = make_int4(e.x, e.y, e.z, claim % H);
+        }
         const uint32_t uslot = k % kUnitSlots;
         if (!(ok = wait_warp(bar(Lay::kUnitEmpty + uslot), ((k / kUnitSlots) & 1) ^ 1, ctl))) break;
         if (lane == 0) {
-          unit_ring[uslot] = u;
+          unit_ring[uslot] = uw;
           ptx::mbar_arrive(bar(Lay::kUnitFull + uslot));
         }
         __syncwarp();
-        if (u < 0) break;
-        const UnitInfo ui = decode_unit(p.work, u, H, causal);
+        if (uw.y < 0) break;
+        const UnitInfo ui = decode_unit(uw, causal);
         if (!(ok = wait_warp(bar(Lay::kQEmpty), (q_it & 1) ^ 1, ctl))) break;
         const int qrow0 = ui.doc_start + kBlockM * ui.qb;
         if constexpr (kFp8) {
@@ -636,12 +707,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         __syncwarp();
         ++q_it;
-        // ring order = consumption order: K_0, K_1, then V_j, K_{j+2}
+        // ring order = consumption order: K_0, K_1, then per step V_j and
+        // K_{j+2} (bf16: K_{j+2} first, its score product is issued first)
         if (!(ok = load_kv(ui, 0, 0))) break;
         if (ui.n > 1 && !(ok = load_kv(ui, 1, 0))) break;
         for (int j = 0; ok && j < ui.n; ++j) {
+          if (Lay::kSepP && j + 2 < ui.n && !(ok = load_kv(ui, j + 2, 0))) break;
           if (!(ok = load_kv(ui, j, 1))) break;
-          if (j + 2 < ui.n && !(ok = load_kv(ui, j + 2, 0))) break;
+          if (!Lay::kSepP && j + 2 < ui.n && !(ok = load_kv(ui, j + 2, 0))) break;
         }
       }
       if (!ok && lane == 0) {
@@ -670,19 +743,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (uint32_t k = 0; ok; ++k) {
         const uint32_t uslot = k % kUnitSlots;
         if (!(ok = wait_one(bar(Lay::kUnitFull + uslot), (k / kUnitSlots) & 1, ctl))) break;
-        const int u = unit_ring[uslot];
+        const int4 uw = unit_ring[uslot];
         ptx::mbar_arrive(bar(Lay::kUnitEmpty + uslot));
-        if (u < 0) break;
-        const UnitInfo ui = decode_unit(p.work, u, H, causal);
+        if (uw.y < 0) break;
+        const UnitInfo ui = decode_unit(uw, causal);
         const int n = ui.n;
         if (!(ok = wait_one(bar(Lay::kQFull), q_ph, ctl))) break;
         q_ph ^= 1;
         ptx::tc_fence_after();
         if constexpr (kFp8)
           tmem_cp_32x128b_x4(tmem + Lay::kTmemSfa, sf_copy_desc(sbase + Lay::kSfaOff));
-        // S for global step gs from the K tile in ring stage st
-        auto score = [&](uint32_t gs, uint32_t st) {
+        // S for global step gs from the K tile in ring stage st; false if a
+        // wait gave up.  bf16: the score buffer must have been read by the
+        // softmax (step gs - 2) first; MXFP8: the in-order issue after
+        // P_{gs-2} V_{gs-2} protects it.
+        auto score = [&](uint32_t gs, uint32_t st) -> bool {
           const uint32_t buf = gs & 1;
+          if constexpr (Lay::kSepP) {
+            if (!wait_one(bar(Lay::kSFree + buf), ((gs >> 1) & 1) ^ 1, ctl)) return false;
+            ptx::tc_fence_after();
+          }
           const uint32_t b_lo = ring_lo + st * (Lay::kSlotBytes >> 4);
           if constexpr (kFp8) {
             const uint32_t sfb = tmem + Lay::kTmemSfb + 4 * buf;
@@ -706,6 +786,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           ptx::mma_commit(bar(Lay::kSFull + buf));
           ptx::mma_commit(bar(Lay::kKVEmpty + st));
+          return true;
         };
         // Next ring tile (in load order); false if the wait gave up.
         auto take = [&](uint32_t& st) -> bool {
@@ -717,36 +798,47 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           return r2;
         };
+        // O += P_j V_j with P_j in TMEM at p_col (+ 8 columns per 16 keys)
+        auto pv = [&](int j, uint32_t st_v, uint32_t buf) {
+          const uint32_t b_lo = ring_lo + st_v * (Lay::kSlotBytes >> 4) + v_lbo;
+#pragma unroll
+          for (int kk = 0; kk < kBlockN / 16; ++kk) {
+            const uint32_t a_col = Lay::kSepP ? Lay::kTmemP + buf * (kBlockN / 2) + kk * 8
+                                              : buf * 128 + (kk >> 2) * kHalfKeys + (kk & 3) * 8;
+            ptx::mma_f16_ts(tmem + Lay::kTmemO, tmem + a_col,
+                            ptx::sdesc_join(b_lo + kk * (2048 >> 4), kDescHi), kIdescO,
+                            (j == 0 && kk == 0) ? 0u : 1u);
+          }
+          ptx::mma_commit(bar(Lay::kKVEmpty + st_v));
+          ptx::mma_commit(bar(Lay::kPFree + buf));
+          if (j == n - 1) ptx::mma_commit(bar(Lay::kOUnit));
+        };
         uint32_t st_k, st_v;
-        if (!(ok = take(st_k))) break;
-        score(g, st_k);
+        if (!(ok = take(st_k)) || !(ok = score(g, st_k))) break;
         if (n > 1) {
-          if (!(ok = take(st_k))) break;
-          score(g + 1, st_k);
+          if (!(ok = take(st_k)) || !(ok = score(g + 1, st_k))) break;
         }
         if (n <= 2) ptx::mma_commit(bar(Lay::kQEmpty));
         for (int j = 0; j < n; ++j) {
           const uint32_t gs = g + j;
           const uint32_t buf = gs & 1;
+          // bf16: S_{j+2} as soon as its buffer is free, ahead of P_j V_j
+          if (Lay::kSepP && j + 2 < n) {
+            if (!(ok = take(st_k)) || !(ok = score(gs + 2, st_k))) break;
+            if (j + 2 == n - 1) ptx::mma_commit(bar(Lay::kQEmpty));
+          }
           if (!(ok = take(st_v))) break;
           if (!(ok = wait_one(bar(Lay::kPFull + buf), (gs >> 1) & 1, ctl))) break;
           if (j == 0 && !(ok = wait_one(bar(Lay::kOEmpty), (oe_cnt++ & 1) ^ 1, ctl))) break;
           ptx::tc_fence_after();
-          const uint32_t b_lo = ring_lo + st_v * (Lay::kSlotBytes >> 4) + v_lbo;
-#pragma unroll
-          for (int kk = 0; kk < kBlockN / 16; ++kk)
-            ptx::mma_f16_ts(tmem + Lay::kTmemO,
-                            tmem + buf * 128 + (kk >> 2) * kHalfKeys + (kk & 3) * 8,
-                            ptx::sdesc_join(b_lo + kk * (2048 >> 4), kDescHi), kIdescO,
-                            (j == 0 && kk == 0) ? 0u : 1u);
-          ptx::mma_commit(bar(Lay::kOFull));
-          ptx::mma_commit(bar(Lay::kKVEmpty + st_v));
-          if (j + 2 < n) {
-            if (!(ok = take(st_k))) break;
-            score(gs + 2, st_k);
+          pv(j, st_v, buf);
+          // MXFP8: S_{j+2} overwrites P_j, so it follows P_j V_j
+          if (!Lay::kSepP && j + 2 < n) {
+            if (!(ok = take(st_k)) || !(ok = score(gs + 2, st_k))) break;
             if (j + 2 == n - 1) ptx::mma_commit(bar(Lay::kQEmpty));
           }
         }
+        if (!ok) break;
         g += n;
       }
       // Every product this thread issued must be complete before TMEM is freed.

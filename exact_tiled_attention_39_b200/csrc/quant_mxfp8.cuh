@@ -16,7 +16,9 @@
 // (an exact power-of-two product) converted by the hardware's
 // round-to-nearest-even, saturating E4M3 conversion.
 //
-// HBM-bound: each thread reads one 64-byte block and writes 32 + 1 bytes.
+// HBM-bound: each thread reads one 64-byte block and writes what the
+// consumer needs: 32 + 1 bytes of codes and scale and/or 64 bytes of exact
+// dequantised bf16.
 #pragma once
 #include <cuda_fp16.h>
 
@@ -59,15 +61,14 @@ __device__ __forceinline__ void e4m3x2_to_f32(uint16_t v, float& lo, float& hi) 
   hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
 }
 
-// One thread per 32-element block; n_blocks = rows * cols / 32.  When `deq`
-// is not null the exact dequantised values (E4M3 value * 2^(code - 127)) are
-// also written as bf16: a 4-bit significand times a power of two is exact in
-// bf16 over the whole range the scale rule produces.
-__global__ void __launch_bounds__(256)
-quantize_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ codes,
-                      uint8_t* __restrict__ scales, uint4* __restrict__ deq, long long n_blocks) {
-  const long long b = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (b >= n_blocks) return;
+// One 32-element block: E4M3 codes and the E8M0 scale, and/or the exact
+// dequantised values (E4M3 value * 2^(code - 127)) as bf16: a 4-bit
+// significand times a power of two is exact in bf16 over the whole range the
+// scale rule produces.  Any of codes, scales and deq may be null (not
+// written).
+__device__ __forceinline__ void quantize_block(const uint4* __restrict__ x, uint4* __restrict__ codes,
+                                               uint8_t* __restrict__ scales, uint4* __restrict__ deq,
+                                               long long b) {
   uint4 v[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) v[i] = x[4 * b + i];
@@ -87,9 +88,11 @@ quantize_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ codes,
     const uint16_t c = cvt_e4m3x2(bf16_lo(w[2 * i + 1]) * inv, bf16_hi(w[2 * i + 1]) * inv);
     out[i] = static_cast<uint32_t>(a) | (static_cast<uint32_t>(c) << 16);
   }
-  codes[2 * b] = make_uint4(out[0], out[1], out[2], out[3]);
-  codes[2 * b + 1] = make_uint4(out[4], out[5], out[6], out[7]);
-  scales[b] = static_cast<uint8_t>(code);
+  if (codes != nullptr) {
+    codes[2 * b] = make_uint4(out[0], out[1], out[2], out[3]);
+    codes[2 * b + 1] = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+  if (scales != nullptr) scales[b] = static_cast<uint8_t>(code);
   if (deq != nullptr) {
     // 2^(code - 127); code 0 needs 2^-127 (subnormal)
     const float mul = code == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(code << 23);
@@ -105,6 +108,36 @@ quantize_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ codes,
 #pragma unroll
     for (int i = 0; i < 4; ++i) deq[4 * b + i] = make_uint4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
   }
+}
+
+// One thread per 32-element block; n_blocks = rows * cols / 32.
+__global__ void __launch_bounds__(256)
+quantize_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ codes,
+                      uint8_t* __restrict__ scales, uint4* __restrict__ deq, long long n_blocks) {
+  const long long b = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b >= n_blocks) return;
+  quantize_block(x, codes, scales, deq, b);
+}
+
+// Q, K and V of one attention call in one launch (blockIdx.y picks the
+// tensor), each with the outputs its consumer reads.
+struct QuantJob {
+  const uint4* x;
+  uint4* codes;
+  uint8_t* scales;
+  uint4* deq;
+};
+struct QuantJobs {
+  QuantJob t[3];
+  long long n_blocks;   // per tensor
+};
+
+__global__ void __launch_bounds__(256)
+quantize_mxfp8_qkv_kernel(const __grid_constant__ QuantJobs jobs) {
+  const long long b = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b >= jobs.n_blocks) return;
+  const QuantJob& j = jobs.t[blockIdx.y];
+  quantize_block(j.x, j.codes, j.scales, j.deq, b);
 }
 
 }  // namespace attn

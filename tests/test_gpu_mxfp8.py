@@ -124,3 +124,29 @@ def test_mxfp8_full_workload_sampled():
     assert e.max() <= MXFP8_MAX_ABS, e.max()
     assert np.abs(lse[heads, toks].double().numpy() - rl).max() <= LSE_ABS
     assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+
+
+def test_mxfp8_repeat_runs_bit_identical():
+    """Repeated runs of the whole MXFP8 path (quantisation pre-pass and the
+    block-scaled kernel) agree bit for bit: each row is computed by one CTA in
+    a fixed order."""
+    inp = workloads.make_inputs("mxfp8_packed")
+    dev = torch.device("cuda:0")
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    cu = inp["cu_seqlens"].to(dev)
+    T, H, d = q.shape
+    ms = max(inp["lengths"])
+    ws = A.make_workspace(A.Shape(T, len(inp["lengths"]), H, d, ms), A.ATTN_MXFP8, dev)
+    first = None
+    for _ in range(3):
+        out = torch.full_like(q, float("nan"))
+        lse = torch.full((H, T), float("nan"), dtype=torch.float32, device=dev)
+        A.attn_fwd(q, k, v, cu, out, lse, True, inp["scale"], dtype=A.ATTN_MXFP8,
+                   workspace=ws, max_seqlen=ms)
+        torch.cuda.synchronize()
+        assert A.attn_get_device_error(ws) == 0
+        if first is None:
+            first = (out.clone(), lse.clone())
+        else:
+            assert torch.equal(out.view(torch.int16), first[0].view(torch.int16))
+            assert torch.equal(lse.view(torch.int32), first[1].view(torch.int32))
