@@ -45,6 +45,41 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def kernel_sources_sha256() -> str:
+    """Hash of the CUDA sources the library is built from (names and bytes)."""
+    import hashlib
+    d = os.path.join(ROOT, "exact_tiled_attention_39_b200", "csrc")
+    h = hashlib.sha256()
+    for n in sorted(os.listdir(d)):
+        if n.endswith((".cu", ".cuh")):
+            h.update(n.encode())
+            with open(os.path.join(d, n), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes (read + write) per attention-kernel launch from the committed
+    ncu summary of this workload, or None when there is none or it was taken
+    on other kernel sources."""
+    p = os.path.join(ROOT, "profiles", f"attn_fwd_kernel_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            line = line.strip().strip("`")
+            for key in ("kernel_sources_sha256", "dram_bytes_per_launch"):
+                if line.startswith(key + ":"):
+                    vals[key] = line.split(":", 1)[1].strip()
+    if vals.get("kernel_sources_sha256") != kernel_sources_sha256():
+        return None
+    try:
+        return int(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -170,17 +205,19 @@ def bench_ours(args):
     err = A.attn_get_device_error(ws)
     value = world * flops / (ms_step * 1e-3) / 1e12
 
-    # ---- per-launch timing of the step on its own stream (roofline)
-    per = []
+    # ---- the attention kernel alone (roofline): CUDA events the library
+    # records on the launching stream around that kernel inside attn_fwd
+    A.attn_timing_enable(True)
+    per, pre = [], []
     for _ in range(5):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
         step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        per.append(e0.elapsed_time(e1))
+        a_ms, p_ms = A.attn_timing_read()
+        per.append(a_ms)
+        pre.append(p_ms)
+    A.attn_timing_enable(False)
+    torch.cuda.synchronize(dev)
     per_ms = statistics.median(per)
+    pre_ms = statistics.median(pre)
 
     # ---- end to end through the public API: pinned host in, host out
     hq, hk, hv = (inp[n].pin_memory() for n in ("q", "k", "v"))
@@ -258,8 +295,11 @@ def bench_ours(args):
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
             "peak_source": f"{peak_source_name(peak_key, dtype)} ({peak_src})",
-            "timed_unit": "one attn_fwd call (schedule kernel + attention kernel), median of 5",
-            "traffic": None,
+            "timed_unit": "attention kernel alone (CUDA events around its launch), median of 5",
+            "kernel_ms": round(per_ms, 4),
+            "prepass_ms": round(pre_ms, 4),
+            "traffic": recorded_traffic(w.name),
+            "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
         },
         "e2e": {
             "value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2),

@@ -13,8 +13,9 @@ from dataclasses import dataclass
 import torch
 
 __all__ = ["ATTN_BF16", "ATTN_MXFP8", "AttnError", "lib", "workspace_size", "attn_fwd",
-           "attn_quantize_mxfp8", "attn_get_device_error", "status_string", "make_workspace",
-           "LIB_PATH", "EXPORTED_SYMBOLS"]
+           "attn_fwd_noalloc", "attn_quantize_mxfp8", "attn_get_device_error", "status_string",
+           "make_workspace", "attn_timing_enable", "attn_timing_read", "LIB_PATH",
+           "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 
@@ -27,7 +28,8 @@ STATUS = {
 }
 
 EXPORTED_SYMBOLS = ("attn_workspace_size", "attn_fwd", "attn_quantize_mxfp8",
-                    "attn_get_device_error", "attn_status_string", "attn_abi_version")
+                    "attn_get_device_error", "attn_status_string", "attn_abi_version",
+                    "attn_fwd_noalloc", "attn_timing_enable", "attn_timing_read")
 
 
 class AttnError(RuntimeError):
@@ -67,6 +69,10 @@ def lib() -> ctypes.CDLL:
         L.attn_status_string.restype = ctypes.c_char_p
         L.attn_abi_version.argtypes = []
         L.attn_abi_version.restype = i32
+        L.attn_timing_enable.argtypes = [i32]
+        L.attn_timing_enable.restype = ctypes.c_int
+        L.attn_timing_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]
+        L.attn_timing_read.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -157,6 +163,23 @@ def attn_quantize_mxfp8(x, codes, scales, stream=None):
                                    _stream_handle(stream, x.device))
     if rc != 0:
         raise AttnError(rc, "attn_quantize_mxfp8")
+
+
+def attn_timing_enable(enable: bool) -> None:
+    """Turn per-call kernel timing on or off (``attn_timing_enable``)."""
+    rc = lib().attn_timing_enable(int(bool(enable)))
+    if rc != 0:
+        raise AttnError(rc, "attn_timing_enable")
+
+
+def attn_timing_read() -> tuple[float, float]:
+    """(attention kernel ms, pre-pass ms) of the most recent timed call;
+    waits for that call's events (``attn_timing_read``)."""
+    a, b = ctypes.c_float(0.0), ctypes.c_float(0.0)
+    rc = lib().attn_timing_read(ctypes.byref(a), ctypes.byref(b))
+    if rc != 0:
+        raise AttnError(rc, "attn_timing_read")
+    return float(a.value), float(b.value)
 
 
 def attn_get_device_error(workspace, stream=None) -> int:

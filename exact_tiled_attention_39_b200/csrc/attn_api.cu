@@ -17,6 +17,38 @@
 namespace attn {
 namespace {
 
+// Events of the timed call (attn_timing_enable / attn_timing_read).
+struct CallTiming {
+  std::mutex mu;
+  bool enabled = false;
+  bool recorded = false;
+  int device = -1;
+  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};   // call start, kernel start, kernel end
+};
+CallTiming g_timing;
+
+// Records event i of the timed call on `strm` when timing is enabled.
+void timing_mark(int i, cudaStream_t strm) {
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  if (!g_timing.enabled) return;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  if (dev != g_timing.device) {
+    for (auto& e : g_timing.ev)
+      if (e != nullptr) {
+        cudaEventDestroy(e);
+        e = nullptr;
+      }
+    g_timing.device = dev;
+    g_timing.recorded = false;
+  }
+  if (g_timing.ev[i] == nullptr && cudaEventCreate(&g_timing.ev[i]) != cudaSuccess) {
+    g_timing.ev[i] = nullptr;
+    return;
+  }
+  if (cudaEventRecord(g_timing.ev[i], strm) == cudaSuccess && i == 2) g_timing.recorded = true;
+}
+
 constexpr int kMaxDevices = 64;
 constexpr int kScheduleThreads = 1024;
 constexpr int kSortCapacityMax = 16384;                   // 128 KB of keys
@@ -209,6 +241,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* header = reinterpret_cast<int32_t*>(ws);
 
+  timing_mark(0, strm);
   // 1. schedule (validates cu_seqlens, writes the work list and its length)
   const int64_t cap = sort_capacity_for(wl.max_entries);
   build_schedule_kernel<<<1, kScheduleThreads, static_cast<size_t>(cap) * 8, strm>>>(
@@ -264,6 +297,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   fp.k_scales = fp8_kernel ? reinterpret_cast<const uint32_t*>(ws + wl.scales_off[1]) : nullptr;
   fp.total_tokens = s.total_tokens;
   fp.num_heads = s.num_heads;
+  fp.head_groups = head_group_count(s.total_tokens, s.num_heads, s.head_dim, fp8_kernel ? 3 : 4);
   fp.causal = causal;
   fp.scale_log2 = scale * 1.4426950408889634f;
   fp.timeout_ns = kWaitTimeoutNs;
@@ -282,6 +316,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
+  timing_mark(1, strm);
   if (fp8_kernel) {
     cfg.dynamicSmemBytes = FwdLayout<128, true>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, true>, tq, tk, tv, fp);
@@ -292,7 +327,26 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
     cfg.dynamicSmemBytes = FwdLayout<64, false>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<64, false>, tq, tk, tv, fp);
   }
+  timing_mark(2, strm);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_timing_enable(int32_t enable) {
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  g_timing.enabled = enable != 0;
+  g_timing.recorded = false;
+  return ATTN_OK;
+}
+
+attn_status_t attn_timing_read(float* attention_ms, float* prepass_ms) {
+  if (attention_ms == nullptr || prepass_ms == nullptr) return ATTN_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  if (!g_timing.recorded) return ATTN_ERR_INVALID_ARG;
+  if (cudaEventSynchronize(g_timing.ev[2]) != cudaSuccess ||
+      cudaEventElapsedTime(attention_ms, g_timing.ev[1], g_timing.ev[2]) != cudaSuccess ||
+      cudaEventElapsedTime(prepass_ms, g_timing.ev[0], g_timing.ev[1]) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return ATTN_OK;
 }
 
 attn_status_t attn_get_device_error(const void* workspace, void* stream, int32_t* device_status) {

@@ -68,6 +68,7 @@ struct FwdParams {
   const uint32_t* k_scales;
   int total_tokens;
   int num_heads;
+  int head_groups;           // unit order: heads in this many groups (see common.cuh)
   int causal;
   float scale_log2;          // scale * log2(e)
   unsigned long long timeout_ns;
@@ -98,16 +99,10 @@ constexpr int kUnitConsumers = 1 + kSoftmaxWarps + 4;   // MMA thread + softmax 
 #endif
 constexpr int kPolyPairPeriod = ATTN_POLY_PAIR_PERIOD;
 
-// Separate-P path: each softmax half reads the other half's scores from TMEM
-// for the row maximum instead of swapping maxima through shared memory.
-#ifndef ATTN_MAX_FROM_TMEM
-#define ATTN_MAX_FROM_TMEM 0
-#endif
-// bf16: P in buffers of its own (1) or over the scores (0).
+// bf16: P in TMEM buffers of its own (1) or over the scores (0).
 #ifndef ATTN_SEPARATE_P
 #define ATTN_SEPARATE_P 1
 #endif
-constexpr bool kMaxFromTmem = ATTN_MAX_FROM_TMEM != 0;
 
 // 2^f on [0, 1): 1 + f (c1 + f (c2 + f c3)), a minimax fit of the relative
 // error (max 8.6e-5) made by csrc/fit_exp2_poly.py; p(0) = 1 exactly.
@@ -410,6 +405,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::tc_fence_after();
         uint32_t sa[64];
         ptx::tmem_ld_x64(t_s, sa);
+        if constexpr (Lay::kSepP) {
+          // this half's scores are in registers: once both halves are, the
+          // buffer may take S_{j+2}
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar(Lay::kSFree + buf));
+        }
         float s[64];
 #pragma unroll
         for (int q = 0; q < 64; ++q) s[q] = __uint_as_float(sa[q]);
@@ -433,46 +435,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int a = 0; a < 8; ++a) mx[a] = ptx::fmax3(mx[a], s[q + 2 * a], s[q + 2 * a + 1]);
         const float m_half = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        float m_other;
-        if constexpr (Lay::kSepP && kMaxFromTmem) {
-          // The other half's scores stay in TMEM until both halves have read
-          // them (P has buffers of its own), so its maximum is read there.
-          const uint32_t t_x = tmem + lane_off + buf * 128 + (h ^ 1) * kHalfKeys;
-          int limit_x = kHalfKeys;
-          if (diag || (j + 1) * kBlockN > ui.doc_len) {
-            limit_x = ui.doc_len - j * kBlockN;
-            if (diag) limit_x = min(limit_x, r + 1);
-            limit_x -= (h ^ 1) * kHalfKeys;
-          }
-          float mo[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            uint32_t xo[32];
-            ptx::tmem_ld_x32(t_x + cc * 32, xo);
-#pragma unroll
-            for (int q = 0; q < 32; q += 2) {
-              const int kq = cc * 32 + q;
-              const float a0 = kq < limit_x ? __uint_as_float(xo[q]) : -INFINITY;
-              const float a1 = kq + 1 < limit_x ? __uint_as_float(xo[q + 1]) : -INFINITY;
-              mo[(q >> 1) & 3] = ptx::fmax3(mo[(q >> 1) & 3], a0, a1);
-            }
-          }
-          m_other = fmaxf(fmaxf(mo[0], mo[1]), fmaxf(mo[2], mo[3]));
-        } else {
-          float* xm = xmax + buf * 2 * kBlockM;
-          xm[h * kBlockM + r] = m_half;
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(bar(Lay::kXFull + buf));
-          if (!(ok = wait_warp(bar(Lay::kXFull + buf), (g >> 1) & 1, ctl))) break;
-          m_other = xm[(h ^ 1) * kBlockM + r];
-        }
-        if constexpr (Lay::kSepP) {
-          // both halves' scores are in registers: the buffer may take S_{j+2}
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(bar(Lay::kSFree + buf));
-        }
-        const float m_tile = fmaxf(m_half, m_other) * c;
+        float* xm = xmax + buf * 2 * kBlockM;
+        xm[h * kBlockM + r] = m_half;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(Lay::kXFull + buf));
+        if (!(ok = wait_warp(bar(Lay::kXFull + buf), (g >> 1) & 1, ctl))) break;
+        const float m_tile = fmaxf(m_half, xm[(h ^ 1) * kBlockM + r]) * c;
         if (j == 0) {
           m_used = m_tile;
         } else {
@@ -673,8 +641,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         claim = __shfl_sync(0xffffffffu, claim, 0);
         int4 uw = make_int4(0, -1, 0, 0);
         if (claim < n_units) {
-          const int4 e = p.work[claim / H];
-          uw = make_int4(e.x, e.y, e.z, claim % H);
+          // Unit -> (entry, head): groups of heads one after the other, the
+          // first H % n_groups groups one head larger; inside a group entry
+          // major (heaviest first), head minor.
+          const int n_entries = n_units / H;
+          const int base = H / p.head_groups, extra = H % p.head_groups;
+          const int big = n_entries * (base + 1);
+          int rem, gsize, h0;
+          if (claim < extra * big) {
+            const int grp = claim / big;
+            rem = claim - grp * big;
+            gsize = base + 1;
+            h0 = grp * (base + 1);
+          } else {
+            const int c2 = claim - extra * big;
+            const int grp = c2 / (n_entries * base);
+            rem = c2 - grp * (n_entries * base);
+            gsize = base;
+            h0 = extra * (base + 1) + grp * base;
+          }
+          const int4 e = p.work[rem / gsize];
+          uw = make_int4(e.x, e.y, e.z, h0 + rem % gsize);
         }
         const uint32_t uslot = k % kUnitSlots;
         if (!(ok = wait_warp(bar(Lay::kUnitEmpty + uslot), ((k / kUnitSlots) & 1) ^ 1, ctl))) break;

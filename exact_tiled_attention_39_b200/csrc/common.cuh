@@ -24,6 +24,23 @@ constexpr size_t kWsAlign = 256;
 // unnormalised weights stay below 2^kRescaleTau.
 constexpr float kRescaleTau = 8.0f;
 
+// Unit order: heads are taken in groups whose K and V fit this much of the
+// L2 (126 MB, split between the two dies), and all units of one group run
+// before the next group's, heaviest first within the group.  Query tiles of
+// one (document, head) then run at about the same time and each K/V tile is
+// fetched from HBM about once instead of once per query tile.
+constexpr double kL2HeadGroupBytes = 40.0 * 1024 * 1024;
+
+// Number of head groups for a launch: heads per group from the budget above
+// (K bytes + V bytes per head over all tokens), groups as equal as possible.
+inline int head_group_count(int64_t total_tokens, int num_heads, int head_dim, int kv_elem_bytes) {
+  const double per_head = static_cast<double>(total_tokens) * head_dim * kv_elem_bytes;
+  int g_max = per_head > 0 ? static_cast<int>(kL2HeadGroupBytes / per_head) : num_heads;
+  if (g_max < 1) g_max = 1;
+  if (g_max > num_heads) g_max = num_heads;
+  return (num_heads + g_max - 1) / g_max;
+}
+
 // Upper bound of the work-list length: every document contributes
 // ceil(L / 128) <= L / 128 + 1 entries.
 inline int64_t max_work_entries(int64_t total_tokens, int64_t num_seqs) {

@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define ATTN_ABI_VERSION 1
+#define ATTN_ABI_VERSION 2
 
 typedef enum {
   ATTN_BF16 = 0,  /* bf16 operands, bf16 tensor-core products, fp32 softmax   */
@@ -156,6 +156,21 @@ attn_status_t attn_quantize_mxfp8(const void* x, uint8_t* codes, uint8_t* scales
  * if the copy fails. */
 attn_status_t attn_get_device_error(const void* workspace, void* stream,
                                     int32_t* device_status);
+
+/* Kernel timing for benchmarks.  While enabled (process-wide), attn_fwd
+ * records three CUDA events on its stream: at the start of the call, just
+ * before the attention kernel and just after it.  attn_timing_read waits for
+ * the events of the most recent timed call and returns, in milliseconds, the
+ * attention kernel's duration and the duration of the work before it in the
+ * same call (schedule build, MXFP8 pre-pass).  Recording the events ends the
+ * overlap of the attention kernel's prologue with the schedule kernel, so a
+ * timed call can be slightly slower than an untimed one; results are
+ * unaffected.  Timed calls from several host threads at once give undefined
+ * timings.  attn_timing_read returns ATTN_ERR_INVALID_ARG for null pointers
+ * or when no call was timed since timing was enabled, ATTN_ERR_CUDA if the
+ * events fail. */
+attn_status_t attn_timing_enable(int32_t enable);
+attn_status_t attn_timing_read(float* attention_ms, float* prepass_ms);
 
 /* Static, human-readable name of a status code. */
 const char* attn_status_string(attn_status_t status);

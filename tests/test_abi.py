@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_version_and_strings(L):
-    assert L.attn_abi_version() == 1
+    assert L.attn_abi_version() == 2
     assert A.status_string(0) == "ATTN_OK"
     assert A.status_string(5) == "ATTN_ERR_BAD_SEQLENS"
     assert A.status_string(6) == "ATTN_ERR_TIMEOUT"
@@ -85,3 +85,14 @@ def test_quantize_host_checks(L):
     assert L.attn_quantize_mxfp8(None, None, None, 0, 64, None) == 0     # empty: no-op
     assert L.attn_quantize_mxfp8(ctypes.c_void_p(16), ctypes.c_void_p(8), ctypes.c_void_p(16),
                                  4, 64, None) == 3
+
+
+def test_timing_read_without_a_timed_call(L):
+    """attn_timing_read reports INVALID_ARG until a call has been timed
+    (no GPU needed: no call is made)."""
+    import ctypes
+    A.attn_timing_enable(True)
+    a, b = ctypes.c_float(), ctypes.c_float()
+    assert L.attn_timing_read(ctypes.byref(a), ctypes.byref(b)) == 1
+    assert L.attn_timing_read(None, None) == 1
+    A.attn_timing_enable(False)
