@@ -1,0 +1,99 @@
+"""Parity figures of the five configurations, one JSON line each (GPU).
+
+    python tests/parity_report.py
+
+Runs every configuration through the C ABI and compares with the fp64 oracle
+the way the GPU tests do: the tiny config element by element (causal and
+non-causal), the large ones on sampled rows (384 random rows plus every
+document's first, second, 128th, 129th, 256th, 257th and last row, random
+heads), MXFP8 against the oracle on the exactly dequantised inputs.  Prints
+max / mean absolute output error, max absolute lse error and the tolerance
+each is held to.  Test infrastructure, like the oracle it calls.
+"""
+from __future__ import annotations
+
+import json
+import os
+import sys
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, os.path.dirname(HERE))
+sys.path.insert(0, HERE)
+
+from exact_tiled_attention_39_b200 import attn as A  # noqa: E402
+from exact_tiled_attention_39_b200 import workloads  # noqa: E402
+from oracle.attention import ref_attention, ref_attention_rows  # noqa: E402
+from oracle.mxfp8 import dequantize_mxfp8_ref, quantize_mxfp8_ref  # noqa: E402
+from helpers import BF16_MAX_ABS, BF16_MEAN_ABS, LSE_ABS, MXFP8_MAX_ABS, run_gpu  # noqa: E402
+
+
+def sample_rows(lengths, H, n, seed):
+    rng = np.random.default_rng(seed)
+    starts = np.concatenate([[0], np.cumsum(lengths)])
+    toks = set(rng.integers(0, int(starts[-1]), n).tolist())
+    for a, b in zip(starts[:-1], starts[1:]):
+        for off in (0, 1, 127, 128, 255, 256):
+            if a + off < b:
+                toks.add(int(a + off))
+        if b > a:
+            toks.add(int(b - 1))
+    toks = np.array(sorted(toks))
+    return toks, rng.integers(0, H, len(toks))
+
+
+def deq(x):
+    c, s = quantize_mxfp8_ref(x.double().numpy())
+    return dequantize_mxfp8_ref(c, s)
+
+
+def line(name, rows, e, le, max_tol, mean_tol):
+    return {"config": name, "rows_compared": int(rows), "max_abs": float(e.max()),
+            "mean_abs": float(e.mean()), "lse_max_abs": float(le.max()),
+            "tol": {"max_abs": max_tol, "mean_abs": mean_tol, "lse": LSE_ABS},
+            "pass": bool(e.max() <= max_tol and (mean_tol is None or e.mean() <= mean_tol)
+                         and le.max() <= LSE_ABS)}
+
+
+def main():
+    out_lines = []
+    inp = workloads.make_inputs("tiny")
+    for causal in (False, True):
+        out, lse, _ = run_gpu(inp["q"], inp["k"], inp["v"], inp["cu_seqlens"], causal,
+                              inp["scale"])
+        ro, rl = ref_attention(inp["q"].double().numpy(), inp["k"].double().numpy(),
+                               inp["v"].double().numpy(), inp["cu_seqlens"].numpy(), causal,
+                               inp["scale"])
+        e = np.abs(out.double().numpy() - ro)
+        le = np.abs(lse.double().numpy() - rl)
+        out_lines.append(line(f"tiny ({'causal' if causal else 'non-causal'})",
+                              ro.shape[0] * ro.shape[1], e, le, BF16_MAX_ABS, BF16_MEAN_ABS))
+    for name in ("dense_causal", "packed_causal", "long_outlier", "mxfp8_packed"):
+        inp = workloads.make_inputs(name)
+        cu = inp["cu_seqlens"]
+        fp8 = name.startswith("mxfp8")
+        out, lse, _ = run_gpu(inp["q"], inp["k"], inp["v"], cu, True, inp["scale"],
+                              dtype=A.ATTN_MXFP8 if fp8 else A.ATTN_BF16,
+                              max_seqlen=max(inp["lengths"]))
+        toks, heads = sample_rows(inp["lengths"], inp["q"].shape[1], 384, seed=1)
+        if fp8:
+            q, k, v = deq(inp["q"]), deq(inp["k"]), deq(inp["v"])
+        else:
+            q, k, v = (inp[n].double().numpy() for n in ("q", "k", "v"))
+        ro, rl = ref_attention_rows(q, k, v, cu.numpy(), True, inp["scale"], toks, heads)
+        e = np.abs(out[toks, heads].double().numpy() - ro)
+        le = np.abs(lse[heads, toks].double().numpy() - rl)
+        out_lines.append(line(name, len(toks), e, le, MXFP8_MAX_ABS if fp8 else BF16_MAX_ABS,
+                              None if fp8 else BF16_MEAN_ABS))
+    for l_ in out_lines:
+        print(json.dumps(l_))
+    return 0 if all(l_["pass"] for l_ in out_lines) else 1
+
+
+if __name__ == "__main__":
+    if not torch.cuda.is_available():
+        print(json.dumps({"skipped": "no CUDA device"}))
+        sys.exit(0)
+    sys.exit(main())
