@@ -9,10 +9,17 @@
 #include <cstring>
 #include <mutex>
 
+#include "attn_fwd_pair_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
 #include "common.cuh"
 #include "quant_mxfp8.cuh"
 #include "schedule.cuh"
+
+// bf16: two query tiles per CTA (attn_fwd_pair_kernel, 1) or one
+// (attn_fwd_kernel, 0).
+#ifndef ATTN_PAIR_KERNEL
+#define ATTN_PAIR_KERNEL 1
+#endif
 
 namespace attn {
 namespace {
@@ -140,6 +147,12 @@ attn_status_t device_info(int* dev_out, DeviceInfo* info) {
         cudaFuncSetAttribute(attn_fwd_kernel<128, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              FwdLayout<128, true>::kBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_pair_kernel<64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PairLayout<64>::kBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_pair_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PairLayout<128>::kBytes) != cudaSuccess ||
         cudaFuncSetAttribute(build_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSortCapacityMax * 8) != cudaSuccess)
       return ATTN_ERR_CUDA;
@@ -241,11 +254,16 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* header = reinterpret_cast<int32_t*>(ws);
 
+  // The block-scaled kernel (MXFP8, d = 128) takes one query tile per unit;
+  // the bf16 kernel two.
+  const bool fp8_kernel = dtype == ATTN_MXFP8 && s.head_dim == 128;
+  const bool pair_kernel = !fp8_kernel && ATTN_PAIR_KERNEL != 0;
   timing_mark(0, strm);
   // 1. schedule (validates cu_seqlens, writes the work list and its length)
   const int64_t cap = sort_capacity_for(wl.max_entries);
   build_schedule_kernel<<<1, kScheduleThreads, static_cast<size_t>(cap) * 8, strm>>>(
-      cu_seqlens, s.num_seqs, s.total_tokens, s.max_seqlen, s.max_seqlen, causal, header,
+      cu_seqlens, s.num_seqs, s.total_tokens, s.max_seqlen, s.max_seqlen, causal,
+      pair_kernel ? 2 : 1, header,
       reinterpret_cast<int4*>(ws + wl.sorted_off), reinterpret_cast<int4*>(ws + wl.unsorted_off),
       static_cast<int>(cap));
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -254,7 +272,6 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   // head-dim elements).  With d = 128 the score product runs block-scaled on
   // the E4M3 codes of q and k, and P V on the exact bf16 dequantisation of v;
   // with d = 64 all three products run on the dequantised values.
-  const bool fp8_kernel = dtype == ATTN_MXFP8 && s.head_dim == 128;
   const void* qk_src[2] = {q, k};
   if (dtype == ATTN_MXFP8) {
     // One launch for all three tensors.  The block-scaled kernel reads the
@@ -311,7 +328,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kFwdThreads);
+  cfg.blockDim = dim3(pair_kernel ? kPairThreads : kFwdThreads);
   cfg.stream = strm;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -320,6 +337,12 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   if (fp8_kernel) {
     cfg.dynamicSmemBytes = FwdLayout<128, true>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, true>, tq, tk, tv, fp);
+  } else if (pair_kernel && s.head_dim == 128) {
+    cfg.dynamicSmemBytes = PairLayout<128>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<128>, tq, tk, tv, fp);
+  } else if (pair_kernel) {
+    cfg.dynamicSmemBytes = PairLayout<64>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<64>, tq, tk, tv, fp);
   } else if (s.head_dim == 128) {
     cfg.dynamicSmemBytes = FwdLayout<128, false>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, false>, tq, tk, tv, fp);

@@ -1,0 +1,536 @@
+// Exact attention forward for sm_100a, bf16: two query tiles per CTA sharing
+// every K/V tile, one softmax warpgroup per query tile.
+//
+// The method is the one of attn_fwd_sm100.cuh ("FlashAttention và IO"
+// (aihero.vn), sections "Tiling giữ công việc ở gần nơi tính" and "Softmax
+// qua nhiều khối cần thống kê chạy": running maximum m, normaliser l and
+// weighted sum u per query row, rescale by exp(m - m_new), result u / l and
+// the log-sum-exp); the loop order and roles follow "FlashAttention,
+// pelatihan multi-GPU, dan kuantisasi bobot" (section 1: outer loop over
+// query blocks, inner over key/value blocks, a producer issuing asynchronous
+// copies, other warps running the products and the softmax).
+//
+// A work unit is a pair of consecutive 128-row query tiles (A = 2t, B =
+// 2t + 1) of one document and head.  Both tiles use the same K_j, V_j, so
+// each K/V tile is loaded once per 256 query rows, and while one tile's
+// softmax works the tensor core runs the other tile's products: per key
+// step the tensor pipe sees P_A V_j, S_A(j+1), P_B V_j, S_B(j+1).
+//
+//   warps 0..3    softmax of tile A (192 registers): one thread per query
+//                 row reads its 128 scores from TMEM, masks, updates m and l,
+//                 writes P (bf16) over the first 64 columns of its scores and
+//                 rescales O_A when the row maximum grew by more than 2^8.
+//   warps 4..7    softmax of tile B.
+//   warps 8..11   epilogue (64 registers): O_t / l_round -> bf16, lse.
+//   warp 12       producer (64 registers): claims units, TMA loads of Q_A,
+//                 Q_B and of K_j, V_j into a ring of shared-memory slots.
+//   warp 13       MMA issuer (one thread).
+//   warps 14..15  idle.
+//
+// TMEM (512 columns, lane = query row): S_A at 0, S_B at 128, O_A at 256,
+// O_B at 384.  S_t(j+1) is issued after P_t V_j has read P_t(j) (in issue
+// order, which the tensor pipe keeps), and its completion also tells the
+// softmax that O_t is up to date for a rescale.
+#pragma once
+#include "attn_fwd_sm100.cuh"
+
+namespace attn {
+
+constexpr int kPairThreads = 512;
+constexpr uint32_t kPairRegsSoftmax = 192, kPairRegsEpilogue = 64, kPairRegsOther = 64;
+static_assert(2 * kPairRegsSoftmax + kPairRegsEpilogue + kPairRegsOther == 4 * 128,
+              "register split must use exactly the registers the CTA is launched with");
+constexpr int kPairUnitConsumers = 1 + 8 + 4;   // MMA thread + softmax warps + epilogue warps
+
+template <int D>
+struct PairLayout {
+  static_assert(D == 64 || D == 128, "head dim 64 or 128");
+  static constexpr int kChunks = D / 64;                      // 128-byte chunks per row
+  static constexpr int kChunkBytes = kBlockM * 128;           // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kChunks * kChunkBytes;    // one Q, K or V tile
+  static constexpr int kQOff = 0;                             // Q_A, then Q_B
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kReserve = 3072;                       // stats, barriers, unit ring
+  static constexpr int kStagesFit = (232448 - kRingOff - kReserve) / kTileBytes;
+  static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
+  static constexpr int kStatsOff = kRingOff + kStages * kTileBytes;   // float [tile][2][128]
+  static constexpr int kBarOff = kStatsOff + 2 * 2 * kBlockM * 4;
+  static constexpr int kQFull = 0, kQEmpty = 1;
+  static constexpr int kKVFull = 2;                           // + stage
+  static constexpr int kKVEmpty = kKVFull + kStages;          // + stage
+  static constexpr int kSFull = kKVEmpty + kStages;           // + tile
+  static constexpr int kPFull = kSFull + 2;                   // + tile
+  static constexpr int kOUnit = kPFull + 2;                   // + tile: O of a unit complete
+  static constexpr int kOEmpty = kOUnit + 2;                  // + tile
+  static constexpr int kStFull = kOEmpty + 2;                 // + tile
+  static constexpr int kStEmpty = kStFull + 2;                // + tile
+  static constexpr int kDrain = kStEmpty + 2;
+  static constexpr int kUnitFull = kDrain + 1;                // + slot
+  static constexpr int kUnitEmpty = kUnitFull + kUnitSlots;   // + slot
+  static constexpr int kNumBars = kUnitEmpty + kUnitSlots;
+  static constexpr int kMiscOff = (kBarOff + kNumBars * 8 + 15) / 16 * 16;   // tmem base, abort
+  static constexpr int kUnitOff = kMiscOff + 16;              // int4 [kUnitSlots]
+  static constexpr int kBytes = kUnitOff + 16 * kUnitSlots;
+  static_assert(kStages >= 3, "too few K/V stages");
+  static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
+  static_assert(kBytes - kStatsOff <= kReserve, "reserve too small");
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmemO = 256;                     // + 128 * tile
+};
+
+// Key steps of query tile qb of a document of doc_len tokens (0 if the tile
+// starts past the document's end).
+__device__ __forceinline__ int tile_steps(int qb, int doc_len, int causal) {
+  if (qb * kBlockM >= doc_len) return 0;
+  const int kv = (doc_len + kBlockN - 1) / kBlockN;
+  return causal ? min(qb + 1, kv) : kv;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPairThreads, 1)
+attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using Lay = PairLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = ptx::smem_addr(smem);
+  if ((sbase & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicCAS(p.err, 0, (int)ATTN_ERR_UNSUPPORTED);
+    return;
+  }
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  auto bar = [&](int i) -> uint32_t { return sbase + Lay::kBarOff + 8 * i; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
+  volatile uint32_t* abort_flag = tmem_holder + 1;
+  float* stats = reinterpret_cast<float*>(smem + Lay::kStatsOff);   // [tile][lse2, 1/l_round][row]
+  int4* unit_ring = reinterpret_cast<int4*>(smem + Lay::kUnitOff);
+
+  constexpr int kWarpTma = 12, kWarpMma = 13;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar(Lay::kQFull), 1);
+    ptx::mbar_init(bar(Lay::kQEmpty), 1);
+    for (int s = 0; s < Lay::kStages; ++s) {
+      ptx::mbar_init(bar(Lay::kKVFull + s), 1);
+      ptx::mbar_init(bar(Lay::kKVEmpty + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      ptx::mbar_init(bar(Lay::kSFull + t), 1);
+      ptx::mbar_init(bar(Lay::kPFull + t), 4);     // the tile's softmax warps
+      ptx::mbar_init(bar(Lay::kOUnit + t), 1);
+      ptx::mbar_init(bar(Lay::kOEmpty + t), 4);    // epilogue warps
+      ptx::mbar_init(bar(Lay::kStFull + t), 4);
+      ptx::mbar_init(bar(Lay::kStEmpty + t), 4);
+    }
+    ptx::mbar_init(bar(Lay::kDrain), 1);
+    for (int i = 0; i < kUnitSlots; ++i) {
+      ptx::mbar_init(bar(Lay::kUnitFull + i), 1);
+      ptx::mbar_init(bar(Lay::kUnitEmpty + i), kPairUnitConsumers);
+    }
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == kWarpTma && lane == 0) {
+    ptx::prefetch_tmap(&tm_q);
+    ptx::prefetch_tmap(&tm_k);
+    ptx::prefetch_tmap(&tm_v);
+  }
+  if (warp == kWarpMma) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_holder), Lay::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  // The work list is written by the schedule-build kernel launched just
+  // before; everything above overlapped with its tail.
+  ptx::grid_dependency_wait();
+
+  const WaitCtl ctl{abort_flag, p.err, p.timeout_ns};
+  const int H = p.num_heads;
+  const int causal = p.causal;
+  auto next_unit_warp = [&](uint32_t k, bool& ok) -> int4 {
+    const uint32_t slot = k % kUnitSlots;
+    if (!(ok = wait_warp(bar(Lay::kUnitFull + slot), (k / kUnitSlots) & 1, ctl)))
+      return make_int4(0, -1, 0, 0);
+    const int4 w = unit_ring[slot];   // after the wait (asm with a memory clobber)
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(bar(Lay::kUnitEmpty + slot));
+    return w;
+  };
+
+  if (warp < 8) {
+    // ------------------------------------------------------------ softmax
+    ptx::regs_increase<kPairRegsSoftmax>();
+    const int t = warp >> 2;                       // query tile of the pair
+    const int r = (warp & 3) * 32 + lane;          // row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + t * 128;
+    const uint32_t t_o = tmem + lane_off + Lay::kTmemO + t * 128;
+    const float c = p.scale_log2;
+    const uint64_t c2 = ptx::f2_pack(c, c);
+    uint32_t g = 0, st_cnt = 0;                    // this tile's key steps, units handed over
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      const int4 uw = next_unit_warp(k, ok);
+      if (uw.y < 0) break;
+      const int doc_len = uw.y;
+      const int qb = 2 * uw.z + t;
+      const int n = tile_steps(qb, doc_len, causal);
+      if (n == 0) continue;
+      float m_used = -INFINITY;   // running maximum in log2 units
+      float l = 0.f;              // sum of the weights
+      float l_round = 0.f;        // sum of the weights as rounded to bf16
+      for (int j = 0; j < n; ++j, ++g) {
+        if (!(ok = wait_warp(bar(Lay::kSFull + t), g & 1, ctl))) break;
+        ptx::tc_fence_after();
+        float s[128];
+        {
+          uint32_t sa[64];
+          ptx::tmem_ld_x64(t_s, sa);
+#pragma unroll
+          for (int q = 0; q < 64; ++q) s[q] = __uint_as_float(sa[q]);
+          ptx::tmem_ld_x64(t_s + 64, sa);
+#pragma unroll
+          for (int q = 0; q < 64; ++q) s[64 + q] = __uint_as_float(sa[q]);
+        }
+        const bool diag = causal && j == qb;
+        if (diag || (j + 1) * kBlockN > doc_len) {
+          int limit = doc_len - j * kBlockN;
+          if (diag) limit = min(limit, r + 1);
+#pragma unroll
+          for (int q = 0; q < 128; ++q)
+            if (q >= limit) s[q] = -INFINITY;
+        }
+        float mx[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx[a] = fmaxf(s[2 * a], s[2 * a + 1]);
+#pragma unroll
+        for (int q = 16; q < 128; q += 16)
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx[a] = ptx::fmax3(mx[a], s[q + 2 * a], s[q + 2 * a + 1]);
+        const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
+        if (j == 0) {
+          m_used = m_tile;
+        } else {
+          // Rescale only rows whose maximum grew past the threshold (warp-wide
+          // TMEM access: other rows take part with a factor of exactly 1).
+          // S_t(j) completed after P_t V_{j-1}, so O_t is up to date.
+          const bool need = m_tile > m_used + kRescaleTau;
+          if (__any_sync(0xffffffffu, need)) {
+            const float m_next = need ? m_tile : m_used;
+            const float alpha = need ? ptx::ex2_approx(m_used - m_next) : 1.f;
+#pragma unroll
+            for (int cc = 0; cc < D / 16; ++cc) {
+              uint32_t o[16];
+              ptx::tmem_ld_x16(t_o + cc * 16, o);
+#pragma unroll
+              for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+              ptx::tmem_st_x16(t_o + cc * 16, o);
+            }
+            l *= alpha;
+            l_round *= alpha;
+            m_used = m_next;
+          }
+        }
+        // Weights rounded to bf16 for the P V product; O is divided by the
+        // sum of the rounded weights, the log-sum-exp uses the exact sum.
+        {
+          const float base = m_used == -INFINITY ? 0.f : m_used;
+          const uint64_t nb2 = ptx::f2_pack(-base, -base);
+          uint64_t se[2];
+          float sr[4];
+#pragma unroll
+          for (int a = 0; a < 2; ++a) se[a] = ptx::f2_pack(0.f, 0.f);
+#pragma unroll
+          for (int a = 0; a < 4; ++a) sr[a] = 0.f;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) {
+              const int q = ch * 16 + kk;
+              const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[2 * q], s[2 * q + 1]), c2, nb2);
+              float x0, x1;
+              ptx::f2_unpack(x, x0, x1);
+              const float p0 = ptx::ex2_approx(x0);
+              const float p1 = ptx::ex2_approx(x1);
+              pk[kk] = ptx::pack_bf16x2(p0, p1);
+              se[kk & 1] = ptx::f2_add(se[kk & 1], ptx::f2_pack(p0, p1));
+              sr[(kk & 1) * 2] = ptx::add_bf16_lo(sr[(kk & 1) * 2], pk[kk]);
+              sr[(kk & 1) * 2 + 1] = ptx::add_bf16_hi(sr[(kk & 1) * 2 + 1], pk[kk]);
+            }
+            ptx::tmem_st_x16(t_s + ch * 16, pk);
+          }
+          float e0, e1;
+          ptx::f2_unpack(ptx::f2_add(se[0], se[1]), e0, e1);
+          l += e0 + e1;
+          l_round += (sr[0] + sr[1]) + (sr[2] + sr[3]);
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(Lay::kPFull + t));
+      }
+      if (!ok) break;
+      if (!(ok = wait_warp(bar(Lay::kStEmpty + t), (st_cnt & 1) ^ 1, ctl))) break;
+      ++st_cnt;
+      stats[(2 * t) * kBlockM + r] = m_used + __log2f(l);
+      stats[(2 * t + 1) * kBlockM + r] = 1.f / l_round;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(Lay::kStFull + t));
+    }
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ epilogue
+    ptx::regs_decrease<kPairRegsEpilogue>();
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    uint32_t st_cnt[2] = {0, 0};
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      const int4 uw = next_unit_warp(k, ok);
+      if (uw.y < 0) break;
+      for (int t = 0; t < 2 && ok; ++t) {
+        const int qb = 2 * uw.z + t;
+        if (tile_steps(qb, uw.y, causal) == 0) continue;
+        const uint32_t cnt = st_cnt[t]++;
+        if (!(ok = wait_warp(bar(Lay::kStFull + t), cnt & 1, ctl))) break;
+        const float lse2 = stats[(2 * t) * kBlockM + r];
+        const float inv_l = stats[(2 * t + 1) * kBlockM + r];
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(Lay::kStEmpty + t));
+        if (!(ok = wait_warp(bar(Lay::kOUnit + t), cnt & 1, ctl))) break;
+        ptx::tc_fence_after();
+        const int row_doc = qb * kBlockM + r;
+        const bool row_ok = row_doc < uw.y;
+        const long long token = static_cast<long long>(uw.x) + row_doc;
+        uint4* orow =
+            reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + (token * H + uw.w) * D);
+        const uint32_t t_o = tmem + (static_cast<uint32_t>(wq * 32) << 16) + Lay::kTmemO + t * 128;
+#pragma unroll
+        for (int cc = 0; cc < D / 16; ++cc) {
+          uint32_t o[16];
+          ptx::tmem_ld_x16(t_o + cc * 16, o);
+          if (cc == D / 16 - 1) {
+            // O_t is in registers: the tensor core may overwrite it now.
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(Lay::kOEmpty + t));
+          }
+          uint32_t w[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            w[q] = ptx::pack_bf16x2(__uint_as_float(o[2 * q]) * inv_l,
+                                    __uint_as_float(o[2 * q + 1]) * inv_l);
+          if (row_ok) {
+            orow[cc * 2] = make_uint4(w[0], w[1], w[2], w[3]);
+            orow[cc * 2 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+          }
+        }
+        if (row_ok)
+          p.lse[static_cast<long long>(uw.w) * p.total_tokens + token] =
+              lse2 * 0.69314718055994530942f;
+      }
+    }
+  } else {
+    ptx::regs_decrease<kPairRegsOther>();
+    if (warp == kWarpTma) {
+      // ---------------------------------------------------------- producer
+      const int n_units = p.ws_header[kWsCountOffset / 4] * H;
+      int* counter = const_cast<int*>(p.ws_header) + kWsUnitCounterOffset / 4;
+      uint32_t q_it = 0, kv_it = 0;
+      bool ok = true;
+      auto load_kv = [&](int head, int row0, const CUtensorMap* tm) -> bool {
+        const uint32_t s = kv_it % Lay::kStages;
+        if (!wait_warp(bar(Lay::kKVEmpty + s), ((kv_it / Lay::kStages) & 1) ^ 1, ctl)) return false;
+        if (lane == 0) {
+          const uint32_t slot = sbase + Lay::kRingOff + s * Lay::kTileBytes;
+          ptx::mbar_arrive_expect_tx(bar(Lay::kKVFull + s), Lay::kTileBytes);
+          for (int cq = 0; cq < Lay::kChunks; ++cq)
+            ptx::tma_load_3d(slot + cq * Lay::kChunkBytes, tm, bar(Lay::kKVFull + s), cq * 64,
+                             head, row0);
+        }
+        __syncwarp();
+        ++kv_it;
+        return true;
+      };
+      for (uint32_t k = 0; ok; ++k) {
+        int claim = 0;
+        if (lane == 0)
+          claim = k == 0 ? static_cast<int>(blockIdx.x)
+                         : static_cast<int>(gridDim.x) + atomicAdd(counter, 1);
+        claim = __shfl_sync(0xffffffffu, claim, 0);
+        int4 uw = make_int4(0, -1, 0, 0);
+        if (claim < n_units) {
+          // Unit -> (entry, head): groups of heads one after the other, the
+          // first H % n_groups groups one head larger; inside a group entry
+          // major (heaviest first), head minor.
+          const int n_entries = n_units / H;
+          const int base = H / p.head_groups, extra = H % p.head_groups;
+          const int big = n_entries * (base + 1);
+          int rem, gsize, h0;
+          if (claim < extra * big) {
+            const int grp = claim / big;
+            rem = claim - grp * big;
+            gsize = base + 1;
+            h0 = grp * (base + 1);
+          } else {
+            const int c2 = claim - extra * big;
+            const int grp = c2 / (n_entries * base);
+            rem = c2 - grp * (n_entries * base);
+            gsize = base;
+            h0 = extra * (base + 1) + grp * base;
+          }
+          const int4 e = p.work[rem / gsize];
+          uw = make_int4(e.x, e.y, e.z, h0 + rem % gsize);
+        }
+        const uint32_t uslot = k % kUnitSlots;
+        if (!(ok = wait_warp(bar(Lay::kUnitEmpty + uslot), ((k / kUnitSlots) & 1) ^ 1, ctl))) break;
+        if (lane == 0) {
+          unit_ring[uslot] = uw;
+          ptx::mbar_arrive(bar(Lay::kUnitFull + uslot));
+        }
+        __syncwarp();
+        if (uw.y < 0) break;
+        const int n_max =
+            max(tile_steps(2 * uw.z, uw.y, causal), tile_steps(2 * uw.z + 1, uw.y, causal));
+        if (!(ok = wait_warp(bar(Lay::kQEmpty), (q_it & 1) ^ 1, ctl))) break;
+        const int qrow0 = uw.x + 2 * kBlockM * uw.z;
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(bar(Lay::kQFull), 2 * Lay::kTileBytes);
+          for (int t = 0; t < 2; ++t)
+            for (int cq = 0; cq < Lay::kChunks; ++cq)
+              ptx::tma_load_3d(sbase + Lay::kQOff + t * Lay::kTileBytes + cq * Lay::kChunkBytes,
+                               &tm_q, bar(Lay::kQFull), cq * 64, uw.w, qrow0 + t * kBlockM);
+        }
+        __syncwarp();
+        ++q_it;
+        // ring order = consumption order: K_0, then V_j, K_{j+1}
+        if (!(ok = load_kv(uw.w, uw.x, &tm_k))) break;
+        for (int j = 0; ok && j < n_max; ++j) {
+          if (!(ok = load_kv(uw.w, uw.x + kBlockN * j, &tm_v))) break;
+          if (j + 1 < n_max && !(ok = load_kv(uw.w, uw.x + kBlockN * (j + 1), &tm_k))) break;
+        }
+      }
+      if (!ok && lane == 0) {
+        // Let copies already issued land before the CTA can exit.
+        WaitCtl drain = ctl;
+        uint32_t zero = 0;
+        drain.abort_flag = &zero;
+        const uint32_t first = kv_it > (uint32_t)Lay::kStages ? kv_it - Lay::kStages : 0;
+        for (uint32_t it = first; it < kv_it; ++it)
+          wait_one(bar(Lay::kKVFull + it % Lay::kStages), (it / Lay::kStages) & 1, drain);
+        if (q_it > 0) wait_one(bar(Lay::kQFull), (q_it - 1) & 1, drain);
+      }
+    } else if (warp == kWarpMma && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t kIdescS = ptx::idesc_bf16(kBlockM, kBlockN, 0);
+      constexpr uint32_t kIdescO = ptx::idesc_bf16(kBlockM, D, 1);
+      constexpr uint32_t kDescHi = ptx::sdesc_hi_sw128(1024);
+      const uint32_t q_lo = ptx::sdesc_lo(sbase + Lay::kQOff, 16);
+      const uint32_t ring_lo = ptx::sdesc_lo(sbase + Lay::kRingOff, 16);
+      const uint32_t v_lbo = static_cast<uint32_t>(Lay::kChunkBytes - 16) >> 4 << 16;
+      uint32_t q_ph = 0;
+      uint32_t g[2] = {0, 0};          // key steps of each tile so far
+      uint32_t oe_cnt[2] = {0, 0};     // units of each tile so far
+      uint32_t cur = 0, cur_ph = 0;    // ring cursor (stage, phase)
+      bool ok = true;
+      auto take = [&](uint32_t& st) -> bool {
+        st = cur;
+        const bool r2 = wait_one(bar(Lay::kKVFull + cur), cur_ph, ctl);
+        if (++cur == static_cast<uint32_t>(Lay::kStages)) {
+          cur = 0;
+          cur_ph ^= 1;
+        }
+        return r2;
+      };
+      // S_t = Q_t K^T with K in ring stage st
+      auto score = [&](int t, uint32_t st) {
+        const uint32_t a_lo = q_lo + ((t * Lay::kTileBytes) >> 4);
+        const uint32_t b_lo = ring_lo + st * (Lay::kTileBytes >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * Lay::kChunkBytes + (kk & 3) * 32) >> 4;
+          ptx::mma_f16_ss(tmem + t * 128, ptx::sdesc_join(a_lo + off, kDescHi),
+                          ptx::sdesc_join(b_lo + off, kDescHi), kIdescS, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(bar(Lay::kSFull + t));
+      };
+      // O_t += P_t V with V in ring stage st
+      auto pv = [&](int t, int j, uint32_t st) {
+        const uint32_t b_lo = ring_lo + st * (Lay::kTileBytes >> 4) + v_lbo;
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk)
+          ptx::mma_f16_ts(tmem + Lay::kTmemO + t * 128, tmem + t * 128 + kk * 8,
+                          ptx::sdesc_join(b_lo + kk * (2048 >> 4), kDescHi), kIdescO,
+                          (j == 0 && kk == 0) ? 0u : 1u);
+      };
+      for (uint32_t k = 0; ok; ++k) {
+        const uint32_t uslot = k % kUnitSlots;
+        if (!(ok = wait_one(bar(Lay::kUnitFull + uslot), (k / kUnitSlots) & 1, ctl))) break;
+        const int4 uw = unit_ring[uslot];
+        ptx::mbar_arrive(bar(Lay::kUnitEmpty + uslot));
+        if (uw.y < 0) break;
+        const int n_t[2] = {tile_steps(2 * uw.z, uw.y, causal), tile_steps(2 * uw.z + 1, uw.y, causal)};
+        const int n_max = max(n_t[0], n_t[1]);
+        if (!(ok = wait_one(bar(Lay::kQFull), q_ph, ctl))) break;
+        q_ph ^= 1;
+        ptx::tc_fence_after();
+        uint32_t st_k, st_v;
+        if (!(ok = take(st_k))) break;
+        for (int t = 0; t < 2; ++t)
+          if (n_t[t] > 0) score(t, st_k);
+        ptx::mma_commit(bar(Lay::kKVEmpty + st_k));
+        if (n_max == 1) ptx::mma_commit(bar(Lay::kQEmpty));
+        for (int j = 0; j < n_max && ok; ++j) {
+          if (!(ok = take(st_v))) break;
+          bool k_taken = false;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= n_t[t]) continue;
+            if (!(ok = wait_one(bar(Lay::kPFull + t), g[t] & 1, ctl))) break;
+            if (j == 0 && !(ok = wait_one(bar(Lay::kOEmpty + t), (oe_cnt[t] & 1) ^ 1, ctl))) break;
+            ptx::tc_fence_after();
+            pv(t, j, st_v);
+            if (j == n_t[t] - 1) {
+              ptx::mma_commit(bar(Lay::kOUnit + t));
+              ++oe_cnt[t];
+            }
+            ++g[t];
+            if (j + 1 < n_t[t]) {
+              if (!k_taken) {
+                if (!(ok = take(st_k))) break;
+                k_taken = true;
+              }
+              score(t, st_k);
+            }
+          }
+          if (!ok) break;
+          ptx::mma_commit(bar(Lay::kKVEmpty + st_v));
+          if (j + 1 < n_max) {
+            if (!k_taken && !(ok = take(st_k))) break;   // unreachable: n_max's tile needs it
+            ptx::mma_commit(bar(Lay::kKVEmpty + st_k));
+            if (j + 2 == n_max) ptx::mma_commit(bar(Lay::kQEmpty));
+          }
+        }
+      }
+      // Every product this thread issued must be complete before TMEM is freed.
+      ptx::mma_commit(bar(Lay::kDrain));
+      WaitCtl drain = ctl;
+      uint32_t zero = 0;
+      drain.abort_flag = &zero;
+      wait_one(bar(Lay::kDrain), 0, drain);
+    }
+  }
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, Lay::kTmemCols);
+  }
+}
+
+}  // namespace attn

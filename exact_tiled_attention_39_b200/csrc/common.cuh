@@ -9,8 +9,9 @@ namespace attn {
 
 constexpr int kBlockM = 128;        // query rows per tile (one TMEM lane per row)
 constexpr int kBlockN = 128;        // keys per key/value tile
-constexpr int kTilesPerUnit = 1;    // query tiles per work unit
-constexpr int kRowsPerUnit = kBlockM * kTilesPerUnit;
+// Work units are 1 query tile (MXFP8 kernel) or 2 (bf16 kernel); the list
+// is sized for the finer granularity.
+constexpr int kRowsPerUnit = kBlockM;
 
 // Workspace layout: a 256-byte header, then the work list.
 constexpr size_t kWsErrorOffset = 0;     // int32 error word (attn_status_t)

@@ -8,10 +8,12 @@
 // pelatihan multi-GPU, dan kuantisasi bobot", section 1 (FlashAttention-2):
 // work is split along the sequence into query blocks.
 //
-// One entry per 128-row query tile of one document:
-// (doc_start, doc_len, query_block, cost), cost = number of key tiles it
-// needs (causal: min(qb + 1, n_kv); else n_kv).  Entries are sorted by cost, largest first, ties in document then
-// pair order, with a bitonic sort of (cost, index) keys in shared memory.
+// One entry per unit of `tiles_per_unit` (1 or 2) consecutive 128-row query
+// tiles of one document: (doc_start, doc_len, unit index, cost), cost = the
+// number of (query tile, key tile) products of its tiles (causal:
+// min(qb + 1, n_kv) per query tile qb; else n_kv).  Entries are sorted by
+// cost, largest first, ties in document then unit order, with a bitonic sort
+// of (cost, index) keys in shared memory.
 #pragma once
 #include <cstdint>
 
@@ -20,12 +22,11 @@
 
 namespace attn {
 
-__device__ __forceinline__ int pair_cost(int L, int t, int causal) {
+__device__ __forceinline__ int unit_cost(int L, int t, int causal, int tiles_per_unit) {
   const int n_kv = (L + kBlockN - 1) / kBlockN;
   int cost = 0;
-#pragma unroll
-  for (int i = 0; i < kTilesPerUnit; ++i) {
-    const int qb = kTilesPerUnit * t + i;
+  for (int i = 0; i < tiles_per_unit; ++i) {
+    const int qb = tiles_per_unit * t + i;
     if (qb * kBlockM < L) cost += causal ? min(qb + 1, n_kv) : n_kv;
   }
   return cost;
@@ -63,7 +64,8 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int* 
 // bytes (sort_capacity a power of two, or 0 to skip sorting).
 __global__ void __launch_bounds__(1024, 1)
 build_schedule_kernel(const int32_t* __restrict__ cu, int num_seqs, int total_tokens,
-                      int max_seqlen, int dense_len, int causal, int32_t* __restrict__ ws_header,
+                      int max_seqlen, int dense_len, int causal, int tiles_per_unit,
+                      int32_t* __restrict__ ws_header,
                       int4* __restrict__ sorted, int4* __restrict__ unsorted, int sort_capacity) {
   extern __shared__ unsigned long long keys[];
   __shared__ int warp_sums[32];
@@ -98,7 +100,7 @@ build_schedule_kernel(const int32_t* __restrict__ cu, int num_seqs, int total_to
     return;
   }
 
-  // 2. enumerate (document, pair) entries in document order
+  // 2. enumerate (document, unit) entries in document order
   int running = 0;
   for (int base = 0; base < num_seqs; base += nt) {
     const int i = base + tid;
@@ -106,10 +108,11 @@ build_schedule_kernel(const int32_t* __restrict__ cu, int num_seqs, int total_to
     if (i < num_seqs) {
       a = cu ? cu[i] : i * dense_len;
       L = cu ? cu[i + 1] - a : dense_len;
-      np = (L + kRowsPerUnit - 1) / kRowsPerUnit;
+      np = (L + kBlockM * tiles_per_unit - 1) / (kBlockM * tiles_per_unit);
     }
     const int first = running + block_exclusive_scan(np, warp_sums, &chunk_total);
-    for (int t = 0; t < np; ++t) unsorted[first + t] = make_int4(a, L, t, pair_cost(L, t, causal));
+    for (int t = 0; t < np; ++t)
+      unsorted[first + t] = make_int4(a, L, t, unit_cost(L, t, causal, tiles_per_unit));
     running += chunk_total;
     __syncthreads();
   }

@@ -1,6 +1,7 @@
-"""Pins of the schedule oracle: hand-worked work lists and the closed-form
-total cost.  CPU only."""
+"""Pins of the schedule oracle: hand-worked work lists (one and two query
+tiles per unit) and the closed-form total cost.  CPU only."""
 import numpy as np
+import pytest
 
 from oracle.schedule import schedule_ref, unit_cost
 
@@ -20,18 +21,29 @@ def test_hand_worked_noncausal():
     np.testing.assert_array_equal(got, np.array(want, dtype=np.int32))
 
 
-def test_total_cost_closed_form():
+def test_hand_worked_pairs():
+    # two query tiles per unit: L=300 has tiles 0,1 | 2; L=400 has 0,1 | 2,3
+    got = schedule_ref([0, 300, 300, 700], causal=True, tiles_per_unit=2)
+    want = [(300, 400, 1, 7), (0, 300, 0, 3), (0, 300, 1, 3), (300, 400, 0, 3)]
+    np.testing.assert_array_equal(got, np.array(want, dtype=np.int32))
+    got = schedule_ref([0, 300, 300, 700], causal=False, tiles_per_unit=2)
+    want = [(300, 400, 0, 8), (300, 400, 1, 8), (0, 300, 0, 6), (0, 300, 1, 3)]
+    np.testing.assert_array_equal(got, np.array(want, dtype=np.int32))
+
+
+@pytest.mark.parametrize("tpu", [1, 2])
+def test_total_cost_closed_form(tpu):
     rng = np.random.default_rng(0)
     lengths = rng.integers(1, 5000, size=40)
     cu = np.concatenate([[0], np.cumsum(lengths)])
     for causal in (False, True):
-        lst = schedule_ref(cu, causal)
+        lst = schedule_ref(cu, causal, tpu)
         n = -(-lengths // 128)
         want = (n * (n + 1) // 2).sum() if causal else (n * n).sum()
         assert int(lst[:, 3].sum()) == int(want)
         assert (np.diff(lst[:, 3]) <= 0).all()
-        # every (doc, query tile) appears once
-        assert len(lst) == int((-(-lengths // 128)).sum())
+        # every (doc, unit) appears once
+        assert len(lst) == int((-(-lengths // (128 * tpu))).sum())
 
 
 def test_unit_cost_edges():
@@ -42,3 +54,8 @@ def test_unit_cost_edges():
     assert unit_cost(256, 0, False) == 2
     assert unit_cost(257, 2, True) == 3
     assert unit_cost(1000, 3, True) == 4
+    # pairs
+    assert unit_cost(1, 0, True, 2) == 1
+    assert unit_cost(129, 0, True, 2) == 3
+    assert unit_cost(256, 0, False, 2) == 4
+    assert unit_cost(257, 1, True, 2) == 3
