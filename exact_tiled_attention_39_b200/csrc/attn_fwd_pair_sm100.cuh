@@ -16,13 +16,13 @@
 // softmax works the tensor core runs the other tile's products: per key
 // step the tensor pipe sees P_A V_j, S_A(j+1), P_B V_j, S_B(j+1).
 //
-//   warps 0..3    softmax of tile A (192 registers): one thread per query
+//   warps 0..3    softmax of tile A (184 registers): one thread per query
 //                 row reads its 128 scores from TMEM, masks, updates m and l,
 //                 writes P (bf16) over the first 64 columns of its scores and
 //                 rescales O_A when the row maximum grew by more than 2^8.
 //   warps 4..7    softmax of tile B.
 //   warps 8..11   epilogue (64 registers): O_t / l_round -> bf16, lse.
-//   warp 12       producer (64 registers): claims units, TMA loads of Q_A,
+//   warp 12       producer (80 registers): claims units, TMA loads of Q_A,
 //                 Q_B and of K_j, V_j into a ring of shared-memory slots.
 //   warp 13       MMA issuer (one thread).
 //   warps 14..15  idle.
@@ -37,7 +37,7 @@
 namespace attn {
 
 constexpr int kPairThreads = 512;
-constexpr uint32_t kPairRegsSoftmax = 192, kPairRegsEpilogue = 64, kPairRegsOther = 64;
+constexpr uint32_t kPairRegsSoftmax = 184, kPairRegsEpilogue = 64, kPairRegsOther = 80;
 static_assert(2 * kPairRegsSoftmax + kPairRegsEpilogue + kPairRegsOther == 4 * 128,
               "register split must use exactly the registers the CTA is launched with");
 constexpr int kPairUnitConsumers = 1 + 8 + 4;   // MMA thread + softmax warps + epilogue warps
