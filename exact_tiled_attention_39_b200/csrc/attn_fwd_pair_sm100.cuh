@@ -253,10 +253,15 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             for (int kk = 0; kk < 16; ++kk) {
               const int q = ch * 16 + kk;
               const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[2 * q], s[2 * q + 1]), c2, nb2);
-              float x0, x1;
+              float x0, x1, p0, p1;
               ptx::f2_unpack(x, x0, x1);
-              const float p0 = ptx::ex2_approx(x0);
-              const float p1 = ptx::ex2_approx(x1);
+              if (kPolyPairPeriod > 0 &&
+                  q % (kPolyPairPeriod > 0 ? kPolyPairPeriod : 1) == kPolyPairPeriod - 1) {
+                exp2_poly_pair(x0, x1, p0, p1);
+              } else {
+                p0 = ptx::ex2_approx(x0);
+                p1 = ptx::ex2_approx(x1);
+              }
               pk[kk] = ptx::pack_bf16x2(p0, p1);
               se[kk & 1] = ptx::f2_add(se[kk & 1], ptx::f2_pack(p0, p1));
               sr[(kk & 1) * 2] = ptx::add_bf16_lo(sr[(kk & 1) * 2], pk[kk]);
