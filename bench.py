@@ -58,11 +58,11 @@ def kernel_sources_sha256() -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, kernel: str):
     """DRAM bytes (read + write) per attention-kernel launch from the committed
-    ncu summary of this workload, or None when there is none or it was taken
-    on other kernel sources."""
-    p = os.path.join(ROOT, "profiles", f"attn_fwd_kernel_{workload}.md")
+    ncu summary of this kernel and workload, or None when there is none or it
+    was taken on other kernel sources."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(p):
         return None
     vals = {}
@@ -267,6 +267,9 @@ def bench_ours(args):
     if dtype == A.ATTN_MXFP8:
         peak *= 2.0        # fp8 dense peak = 2 x bf16 (nominal ratio)
     achieved = flops / (per_ms * 1e-3) / 1e12
+    # bf16 runs the two-query-tile kernel, MXFP8 (head dim 128) the
+    # block-scaled one-tile kernel
+    kernel_name = "attn_fwd_kernel" if dtype == A.ATTN_MXFP8 else "attn_fwd_pair_kernel"
 
     line = {
         "metric": METRIC,
@@ -298,7 +301,8 @@ def bench_ours(args):
             "timed_unit": "attention kernel alone (CUDA events around its launch), median of 5",
             "kernel_ms": round(per_ms, 4),
             "prepass_ms": round(pre_ms, 4),
-            "traffic": recorded_traffic(w.name),
+            "kernel": kernel_name,
+            "traffic": recorded_traffic(w.name, kernel_name),
             "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
         },
         "e2e": {
