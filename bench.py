@@ -80,6 +80,35 @@ def recorded_traffic(workload: str, kernel: str):
         return None
 
 
+def init_group(backend: str, device=None):
+    """Process group over the launcher's ranks (torchrun env, 127.0.0.1
+    rendezvous), or None for one process.  A short timeout makes ranks that
+    wait for a missing peer fail instead of hanging."""
+    world, _, _ = dist_env()
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    kw = {"device_id": device} if backend == "nccl" else {}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    return dist
+
+
+def max_over_ranks(pg, value: float, device) -> float:
+    """The largest of every rank's value (every rank gets it)."""
+    if pg is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world: int, flops_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: every rank runs the same workload (independent
+    replicas), the job takes the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -149,13 +178,7 @@ def bench_ours(args):
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-        pg = dist
+    pg = init_group("nccl", dev)
 
     w = workloads.get(args.workload)
     inp = workloads.make_inputs(w)
@@ -196,14 +219,10 @@ def bench_ours(args):
         torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
-    ms_total = t0.elapsed_time(t1)
-    if pg:
-        tt = torch.tensor([ms_total], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(pg, t0.elapsed_time(t1), dev)
     ms_step = ms_total / args.steps
     err = A.attn_get_device_error(ws)
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(world, flops, ms_step)
 
     # ---- the attention kernel alone (roofline): CUDA events the library
     # records on the launching stream around that kernel inside attn_fwd
@@ -246,11 +265,7 @@ def bench_ours(args):
         e2e_step()
     s1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = s0.elapsed_time(s1) / e2e_steps
-    if pg:
-        tt = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(tt, op=pg.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(pg, s0.elapsed_time(s1) / e2e_steps, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcu))
     d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
 
@@ -306,7 +321,7 @@ def bench_ours(args):
             "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
         },
         "e2e": {
-            "value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2),
+            "value": round(aggregate_tflops(world, flops, e2e_ms), 2),
             "unit": "TFLOP/s",
             "ms_per_step": round(e2e_ms, 3),
             "h2d_bytes_per_step": h2d,
