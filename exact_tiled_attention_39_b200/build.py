@@ -63,5 +63,24 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_variant(name: str, defines: dict[str, str]) -> str:
+    """Build ``libattn_<name>.so`` in-tree with extra preprocessor defines
+    (test builds: the failure-detection test uses one); rebuilt when a source
+    is newer."""
+    out = os.path.join(PKG, f"libattn_{name}.so")
+    deps = sources() + [os.path.join(ROOT, "include", "attn.h"), __file__]
+    if os.path.exists(out) and all(os.path.getmtime(s) <= os.path.getmtime(out) for s in deps):
+        return out
+    cmd = [_nvcc(), *[f for f in NVCC_FLAGS if f not in ("-Xptxas", "-v")],
+           *[f"-D{k}={v}" for k, v in defines.items()], "-I", os.path.join(ROOT, "include"),
+           os.path.join(CSRC, "attn_api.cu"), "-o", out + ".tmp"]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError(f"nvcc failed building libattn_{name}.so")
+    os.replace(out + ".tmp", out)
+    return out
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose=True))

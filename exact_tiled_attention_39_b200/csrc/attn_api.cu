@@ -59,7 +59,12 @@ void timing_mark(int i, cudaStream_t strm) {
 constexpr int kMaxDevices = 64;
 constexpr int kScheduleThreads = 1024;
 constexpr int kSortCapacityMax = 16384;                   // 128 KB of keys
-constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;  // 1 s per wait
+// Limit of every mbarrier wait in the kernels (a build for the failure tests
+// sets a short one).
+#ifndef ATTN_WAIT_TIMEOUT_NS
+#define ATTN_WAIT_TIMEOUT_NS 1000000000ull
+#endif
+constexpr unsigned long long kWaitTimeoutNs = ATTN_WAIT_TIMEOUT_NS;  // 1 s per wait by default
 
 struct DeviceInfo {
   bool ready = false;

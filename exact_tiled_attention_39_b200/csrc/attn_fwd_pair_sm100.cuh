@@ -36,6 +36,14 @@
 
 namespace attn {
 
+// Failure-test build only: the first unit's S_A-ready signal is never sent,
+// so tile A's softmax waits run out, the CTA aborts and the call reports
+// ATTN_ERR_TIMEOUT (with a short ATTN_WAIT_TIMEOUT_NS).
+#ifndef ATTN_FAULT_DROP_FIRST_SCORE_COMMIT
+#define ATTN_FAULT_DROP_FIRST_SCORE_COMMIT 0
+#endif
+constexpr bool kFaultDropFirstScoreCommit = ATTN_FAULT_DROP_FIRST_SCORE_COMMIT != 0;
+
 constexpr int kPairThreads = 512;
 constexpr uint32_t kPairRegsSoftmax = 184, kPairRegsEpilogue = 64, kPairRegsOther = 80;
 static_assert(2 * kPairRegsSoftmax + kPairRegsEpilogue + kPairRegsOther == 4 * 128,
@@ -452,7 +460,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         return r2;
       };
       // S_t = Q_t K^T with K in ring stage st
-      auto score = [&](int t, uint32_t st) {
+      auto score = [&](int t, uint32_t st, bool commit = true) {
         const uint32_t a_lo = q_lo + ((t * Lay::kTileBytes) >> 4);
         const uint32_t b_lo = ring_lo + st * (Lay::kTileBytes >> 4);
 #pragma unroll
@@ -461,7 +469,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           ptx::mma_f16_ss(tmem + t * 128, ptx::sdesc_join(a_lo + off, kDescHi),
                           ptx::sdesc_join(b_lo + off, kDescHi), kIdescS, kk > 0 ? 1u : 0u);
         }
-        ptx::mma_commit(bar(Lay::kSFull + t));
+        if (commit) ptx::mma_commit(bar(Lay::kSFull + t));
       };
       // O_t += P_t V with V in ring stage st
       auto pv = [&](int t, int j, uint32_t st) {
@@ -486,7 +494,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         uint32_t st_k, st_v;
         if (!(ok = take(st_k))) break;
         for (int t = 0; t < 2; ++t)
-          if (n_t[t] > 0) score(t, st_k);
+          if (n_t[t] > 0) score(t, st_k, !(kFaultDropFirstScoreCommit && k == 0 && t == 0));
         ptx::mma_commit(bar(Lay::kKVEmpty + st_k));
         if (n_max == 1) ptx::mma_commit(bar(Lay::kQEmpty));
         for (int j = 0; j < n_max && ok; ++j) {
