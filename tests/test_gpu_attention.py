@@ -276,3 +276,24 @@ def test_repeat_runs_bit_identical(name):
         else:
             assert torch.equal(out.view(torch.int16), first[0].view(torch.int16))
             assert torch.equal(lse.view(torch.int32), first[1].view(torch.int32))
+
+
+def test_many_documents_unsorted_schedule():
+    """18000 one-token documents and three longer ones: more work-list
+    entries than the schedule builder sorts in shared memory (16384), so the
+    list stays in document order; every row is still right (a one-token
+    document's output is its own value row and its lse its own score)."""
+    lengths = [1] * 18000 + [300, 129, 700]
+    q, k, v, cu = _pack(lengths, 1, 64, seed=21)
+    out, lse, ws = run_gpu(q, k, v, cu, True, 0.125, max_seqlen=700)
+    assert A.attn_get_device_error(ws) == 0
+    hdr = ws[:8].cpu().view(torch.int32)
+    assert int(hdr[1]) == 18000 + 2 + 1 + 3        # pairs of query tiles
+    # one-token documents: exact
+    assert torch.equal(out[:18000], v[:18000])
+    s = (q[:18000, 0].double() * k[:18000, 0].double()).sum(-1) * 0.125
+    assert np.abs(lse[0, :18000].double().numpy() - s.numpy()).max() <= 1e-4
+    # the long documents against the oracle
+    sub = slice(18000, None)
+    ro, rl = _oracle(q[sub], k[sub], v[sub], workloads.cu_from_lengths([300, 129, 700]), True, 0.125)
+    _check(out[sub], lse[:, sub], ro, rl, None)
