@@ -385,7 +385,7 @@ def bench_reference(args):
     for _ in range(args.warmup):
         cpu_baseline(w, inp, budget_s=budget)
     vals = [cpu_baseline(w, inp, budget_s=budget) for _ in range(args.steps)]
-    v = statistics.median(x["value"] for x in vals)
+    v = round(statistics.median(x["value"] for x in vals), 6)
     T, H, d = inp["q"].shape
     flops = workloads.flops(inp["lengths"], H, d, True)
     return {
