@@ -15,12 +15,6 @@
 #include "quant_mxfp8.cuh"
 #include "schedule.cuh"
 
-// bf16: two query tiles per CTA (attn_fwd_pair_kernel, 1) or one
-// (attn_fwd_kernel, 0).
-#ifndef ATTN_PAIR_KERNEL
-#define ATTN_PAIR_KERNEL 1
-#endif
-
 namespace attn {
 namespace {
 
@@ -143,13 +137,7 @@ attn_status_t device_info(int* dev_out, DeviceInfo* info) {
   if (!d.ready) {
     if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<64, false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FwdLayout<64, false>::kBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_kernel<128, false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FwdLayout<128, false>::kBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_kernel<128, true>,
+    if (cudaFuncSetAttribute(attn_fwd_kernel<128, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              FwdLayout<128, true>::kBytes) != cudaSuccess ||
         cudaFuncSetAttribute(attn_fwd_pair_kernel<64>,
@@ -262,7 +250,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   // The block-scaled kernel (MXFP8, d = 128) takes one query tile per unit;
   // the bf16 kernel two.
   const bool fp8_kernel = dtype == ATTN_MXFP8 && s.head_dim == 128;
-  const bool pair_kernel = !fp8_kernel && ATTN_PAIR_KERNEL != 0;
+  const bool pair_kernel = !fp8_kernel;
   timing_mark(0, strm);
   // 1. schedule (validates cu_seqlens, writes the work list and its length)
   const int64_t cap = sort_capacity_for(wl.max_entries);
@@ -342,18 +330,12 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   if (fp8_kernel) {
     cfg.dynamicSmemBytes = FwdLayout<128, true>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, true>, tq, tk, tv, fp);
-  } else if (pair_kernel && s.head_dim == 128) {
+  } else if (s.head_dim == 128) {
     cfg.dynamicSmemBytes = PairLayout<128>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<128>, tq, tk, tv, fp);
-  } else if (pair_kernel) {
+  } else {
     cfg.dynamicSmemBytes = PairLayout<64>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<64>, tq, tk, tv, fp);
-  } else if (s.head_dim == 128) {
-    cfg.dynamicSmemBytes = FwdLayout<128, false>::kBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, false>, tq, tk, tv, fp);
-  } else {
-    cfg.dynamicSmemBytes = FwdLayout<64, false>::kBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<64, false>, tq, tk, tv, fp);
   }
   timing_mark(2, strm);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

@@ -1,6 +1,9 @@
-// Exact attention forward for sm_100a: persistent, warp-specialised,
-// TMA + tcgen05 + TMEM; bf16 operands, or MXFP8 (E4M3 with E8M0 block scales)
-// for the score product.
+// Exact attention forward for sm_100a, MXFP8: persistent, warp-specialised,
+// TMA + tcgen05 + TMEM, with the score product block-scaled (E4M3 operands,
+// E8M0 scales) and P V in bf16 on the exactly dequantised values.  Also the
+// helpers (bounded waits, unit decode, exponentials) the bf16 kernel in
+// attn_fwd_pair_sm100.cuh uses.  The host instantiates it for head dim 128
+// with MXFP8 operands; the template keeps a bf16 mode (kFp8 = false).
 //
 // The method ("FlashAttention và IO" (aihero.vn), sections "Tiling giữ công
 // việc ở gần nơi tính" and "Softmax qua nhiều khối cần thống kê chạy"):
@@ -13,14 +16,15 @@
 // Loop order and roles follow "FlashAttention, pelatihan multi-GPU, dan
 // kuantisasi bobot" (section 1): outer loop over query blocks, inner over
 // key/value blocks; a producer issues asynchronous tile copies while other
-// warps run the products and the softmax.  The MXFP8 variant follows
+// warps run the products and the softmax.  The MXFP8 products follow
 // "FLAMIA: Blackwell Üzerinde Hızlı ve Nedensel Olarak Güvenli Eğitim İçin
 // Flash Mikro-Ölçeklemeli Dikkat Mekanizması" (section "FLAMIA Mimarisi ve
 // Temel Tasarım İlkeleri"): block-scaled low-precision products whose scales
 // (one per token, head and 32 head-dim elements) never span two tokens.
 //
-// A work unit is one 128-row query tile of one document and head.  On
-// sm_100a (512 threads, registers re-split per warpgroup with setmaxnreg):
+// A work unit is one 128-row query tile of one document and head (the scale
+// factors take the TMEM a second query tile would need).  On sm_100a (512
+// threads, registers re-split per warpgroup with setmaxnreg):
 //
 //   warps 0..7    softmax (168 registers), two warpgroups on the same rows:
 //                 warpgroup h takes keys [64 h, 64 h + 64) of every score
@@ -32,8 +36,8 @@
 //                 more than 2^8 (lazy rescale).
 //   warps 8..11   epilogue (96 registers): O / l to bf16 and the log-sum-exp.
 //   warp 12       producer (80 registers): claims units, TMA loads of Q and of
-//                 K_j, V_j into a ring of shared-memory slots; for MXFP8 the
-//                 whole warp also stages the E8M0 scale blocks.
+//                 K_j, V_j into a ring of shared-memory slots; the whole warp
+//                 also stages the E8M0 scale blocks.
 //   warp 13       MMA issuer (one thread): S = Q K_j^T into one of two TMEM
 //                 score buffers, O += P V_j with P read from TMEM.
 //   warps 14..15  idle.
@@ -41,13 +45,12 @@
 // The score buffers alternate between key steps, so while the softmax works
 // on step j the tensor core computes P_{j-1} V_{j-1} and S_{j+1}.  Splitting
 // a row between two warps halves the softmax latency of a step and puts two
-// softmax warps on every SM sub-partition, which keeps the exponential unit
-// fed while the other warp waits on a dependency.
+// softmax warps on every SM sub-partition.
 //
 // TMEM (512 columns, lane = query row): S buffers at columns 0 and 128 (the
 // P half of warpgroup h overwrites columns [64 h, 64 h + 32) of its buffer),
-// O at 256; for MXFP8 the scale factors of Q at 384 and of the current K tile
-// at 388 / 392.
+// O at 256, the scale factors of Q at 384 and of the current K tile at
+// 388 / 392.
 #pragma once
 #include <cuda.h>
 
@@ -99,10 +102,6 @@ constexpr int kUnitConsumers = 1 + kSoftmaxWarps + 4;   // MMA thread + softmax 
 #endif
 constexpr int kPolyPairPeriod = ATTN_POLY_PAIR_PERIOD;
 
-// bf16: P in TMEM buffers of its own (1) or over the scores (0).
-#ifndef ATTN_SEPARATE_P
-#define ATTN_SEPARATE_P 1
-#endif
 
 // 2^f on [0, 1): 1 + f (c1 + f (c2 + f c3)), a minimax fit of the relative
 // error (max 8.6e-5) made by csrc/fit_exp2_poly.py; p(0) = 1 exactly.
@@ -146,8 +145,7 @@ struct FwdLayout {
   static constexpr int kStFull = kOEmpty + 1;
   static constexpr int kStEmpty = kStFull + 1;
   static constexpr int kXFull = kStEmpty + 1;                // + step parity
-  static constexpr int kSFree = kXFull + 2;                   // + buffer (bf16 only)
-  static constexpr int kPFree = kSFree + 2;                   // + buffer: P V of that buffer done
+  static constexpr int kPFree = kXFull + 2;                   // + buffer: P V of that buffer done
   static constexpr int kDrain = kPFree + 2;
   static constexpr int kUnitFull = kDrain + 1;                // + slot
   static constexpr int kUnitEmpty = kUnitFull + kUnitSlots;   // + slot
@@ -159,12 +157,6 @@ struct FwdLayout {
   static_assert(kBytes - kStatsOff <= kReserve, "reserve too small");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemO = 256, kTmemSfa = 384, kTmemSfb = 388;
-  // bf16: P has buffers of its own (64 columns each) after O, so the next
-  // score product can overwrite a score buffer as soon as the softmax has
-  // read it.  MXFP8 needs those columns for the scale factors and writes P
-  // over the scores instead.
-  static constexpr bool kSepP = !kFp8 && ATTN_SEPARATE_P != 0;
-  static constexpr uint32_t kTmemP = 384;
 };
 
 // Bounded waits.  A wait gives up when the CTA's abort flag is raised or
@@ -332,7 +324,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       ptx::mbar_init(bar(Lay::kSFull + b), 1);
       ptx::mbar_init(bar(Lay::kPFull + b), kSoftmaxWarps);   // one arrival per softmax warp
       ptx::mbar_init(bar(Lay::kXFull + b), kSoftmaxWarps);
-      ptx::mbar_init(bar(Lay::kSFree + b), kSoftmaxWarps);
       ptx::mbar_init(bar(Lay::kPFree + b), 1);
     }
     ptx::mbar_init(bar(Lay::kOUnit), 1);
@@ -405,13 +396,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::tc_fence_after();
         uint32_t sa[64];
         ptx::tmem_ld_x64(t_s, sa);
-        if constexpr (Lay::kSepP) {
-          // this half's scores are in registers: once both halves are, the
-          // buffer may take S_{j+2}
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(bar(Lay::kSFree + buf));
-        }
         float s[64];
 #pragma unroll
         for (int q = 0; q < 64; ++q) s[q] = __uint_as_float(sa[q]);
@@ -476,14 +460,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // combination of the values with the weights actually used (no bias
         // from the rounding, which matters when one key dominates a row);
         // l sums the unrounded weights and gives the log-sum-exp.
-        // P of this step goes to its own buffer (bf16) once the P V product
-        // two steps back has read it, else over this half's scores (which
-        // that product has read as well: this step's scores came after it).
-        // The wait is taken on both paths, after the weights are formed; it
-        // also keeps this warp at most one phase behind each buffer's barrier.
-        const uint32_t t_p =
-            Lay::kSepP ? tmem + lane_off + Lay::kTmemP + buf * (kBlockN / 2) + h * (kHalfKeys / 2)
-                       : t_s;
+        // P of this step goes over this half's scores.  The P V product two
+        // steps back has read that buffer already (these scores came after
+        // it); the wait on its barrier, after the weights are formed, keeps
+        // this warp at most one phase behind each buffer's barrier.
+        const uint32_t t_p = t_s;
         {
           const float base = m_used == -INFINITY ? 0.f : m_used;
           const uint64_t nb2 = ptx::f2_pack(-base, -base);
@@ -695,13 +676,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncwarp();
         ++q_it;
         // ring order = consumption order: K_0, K_1, then per step V_j and
-        // K_{j+2} (bf16: K_{j+2} first, its score product is issued first)
+        // K_{j+2}
         if (!(ok = load_kv(ui, 0, 0))) break;
         if (ui.n > 1 && !(ok = load_kv(ui, 1, 0))) break;
         for (int j = 0; ok && j < ui.n; ++j) {
-          if (Lay::kSepP && j + 2 < ui.n && !(ok = load_kv(ui, j + 2, 0))) break;
           if (!(ok = load_kv(ui, j, 1))) break;
-          if (!Lay::kSepP && j + 2 < ui.n && !(ok = load_kv(ui, j + 2, 0))) break;
+          if (j + 2 < ui.n && !(ok = load_kv(ui, j + 2, 0))) break;
         }
       }
       if (!ok && lane == 0) {
@@ -740,16 +720,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::tc_fence_after();
         if constexpr (kFp8)
           tmem_cp_32x128b_x4(tmem + Lay::kTmemSfa, sf_copy_desc(sbase + Lay::kSfaOff));
-        // S for global step gs from the K tile in ring stage st; false if a
-        // wait gave up.  bf16: the score buffer must have been read by the
-        // softmax (step gs - 2) first; MXFP8: the in-order issue after
-        // P_{gs-2} V_{gs-2} protects it.
+        // S for global step gs from the K tile in ring stage st.  It
+        // overwrites P_{gs-2}, so it is issued after P_{gs-2} V_{gs-2} (the
+        // tensor pipe keeps issue order).
         auto score = [&](uint32_t gs, uint32_t st) -> bool {
           const uint32_t buf = gs & 1;
-          if constexpr (Lay::kSepP) {
-            if (!wait_one(bar(Lay::kSFree + buf), ((gs >> 1) & 1) ^ 1, ctl)) return false;
-            ptx::tc_fence_after();
-          }
           const uint32_t b_lo = ring_lo + st * (Lay::kSlotBytes >> 4);
           if constexpr (kFp8) {
             const uint32_t sfb = tmem + Lay::kTmemSfb + 4 * buf;
@@ -785,13 +760,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           return r2;
         };
-        // O += P_j V_j with P_j in TMEM at p_col (+ 8 columns per 16 keys)
+        // O += P_j V_j with P_j in TMEM over the scores: keys 64 h + k of
+        // half h at column 64 h + k / 2 of the buffer
         auto pv = [&](int j, uint32_t st_v, uint32_t buf) {
           const uint32_t b_lo = ring_lo + st_v * (Lay::kSlotBytes >> 4) + v_lbo;
 #pragma unroll
           for (int kk = 0; kk < kBlockN / 16; ++kk) {
-            const uint32_t a_col = Lay::kSepP ? Lay::kTmemP + buf * (kBlockN / 2) + kk * 8
-                                              : buf * 128 + (kk >> 2) * kHalfKeys + (kk & 3) * 8;
+            const uint32_t a_col = buf * 128 + (kk >> 2) * kHalfKeys + (kk & 3) * 8;
             ptx::mma_f16_ts(tmem + Lay::kTmemO, tmem + a_col,
                             ptx::sdesc_join(b_lo + kk * (2048 >> 4), kDescHi), kIdescO,
                             (j == 0 && kk == 0) ? 0u : 1u);
@@ -809,18 +784,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int j = 0; j < n; ++j) {
           const uint32_t gs = g + j;
           const uint32_t buf = gs & 1;
-          // bf16: S_{j+2} as soon as its buffer is free, ahead of P_j V_j
-          if (Lay::kSepP && j + 2 < n) {
-            if (!(ok = take(st_k)) || !(ok = score(gs + 2, st_k))) break;
-            if (j + 2 == n - 1) ptx::mma_commit(bar(Lay::kQEmpty));
-          }
           if (!(ok = take(st_v))) break;
           if (!(ok = wait_one(bar(Lay::kPFull + buf), (gs >> 1) & 1, ctl))) break;
           if (j == 0 && !(ok = wait_one(bar(Lay::kOEmpty), (oe_cnt++ & 1) ^ 1, ctl))) break;
           ptx::tc_fence_after();
           pv(j, st_v, buf);
-          // MXFP8: S_{j+2} overwrites P_j, so it follows P_j V_j
-          if (!Lay::kSepP && j + 2 < n) {
+          // S_{j+2} overwrites P_j, so it follows P_j V_j
+          if (j + 2 < n) {
             if (!(ok = take(st_k)) || !(ok = score(gs + 2, st_k))) break;
             if (j + 2 == n - 1) ptx::mma_commit(bar(Lay::kQEmpty));
           }
