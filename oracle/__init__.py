@@ -11,6 +11,9 @@ Modules
 attention  fp64 attention by its definition (full masked score matrix per
            document and head), the online-softmax recurrence replayed step by
            step, and a per-row evaluator for sampled checks at full size.
+attention_bwd
+           fp64 gradients (dQ, dK, dV) of the same definition, for the
+           backward pass that follows the forward.
 mxfp8      bit-exact E4M3 / E8M0 block quantiser and exact dequantiser.
 schedule   the heaviest-first work list the schedule-build step must emit.
 
