@@ -45,16 +45,28 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# attn_api.cu holds the backward's host code after this line; the forward's
+# sources end before it.
+BWD_SECTION_MARK = b"\n// " + b"=" * 75 + b"\n// Backward (bf16)"
+
+
 def kernel_sources_sha256() -> str:
-    """Hash of the CUDA sources the library is built from (names and bytes)."""
+    """Hash of the CUDA sources the forward kernels are built and launched
+    from (names and bytes): every csrc file except the backward's, and
+    attn_api.cu up to its backward section."""
     import hashlib
     d = os.path.join(ROOT, "exact_tiled_attention_39_b200", "csrc")
     h = hashlib.sha256()
     for n in sorted(os.listdir(d)):
-        if n.endswith((".cu", ".cuh")):
+        if n.endswith((".cu", ".cuh")) and not n.startswith("attn_bwd"):
             h.update(n.encode())
             with open(os.path.join(d, n), "rb") as f:
-                h.update(f.read())
+                data = f.read()
+            if n == "attn_api.cu":
+                cut = data.find(BWD_SECTION_MARK)
+                if cut >= 0:
+                    data = data[:cut]
+            h.update(data)
     return h.hexdigest()
 
 

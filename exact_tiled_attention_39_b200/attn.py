@@ -14,8 +14,8 @@ import torch
 
 __all__ = ["ATTN_BF16", "ATTN_MXFP8", "AttnError", "lib", "workspace_size", "attn_fwd",
            "attn_fwd_noalloc", "attn_quantize_mxfp8", "attn_get_device_error", "status_string",
-           "make_workspace", "attn_timing_enable", "attn_timing_read", "LIB_PATH",
-           "EXPORTED_SYMBOLS"]
+           "make_workspace", "attn_timing_enable", "attn_timing_read", "bwd_workspace_size",
+           "make_bwd_workspace", "attn_bwd", "LIB_PATH", "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 
@@ -29,7 +29,8 @@ STATUS = {
 
 EXPORTED_SYMBOLS = ("attn_workspace_size", "attn_fwd", "attn_quantize_mxfp8",
                     "attn_get_device_error", "attn_status_string", "attn_abi_version",
-                    "attn_fwd_noalloc", "attn_timing_enable", "attn_timing_read")
+                    "attn_fwd_noalloc", "attn_timing_enable", "attn_timing_read",
+                    "attn_bwd_workspace_size", "attn_bwd")
 
 
 class AttnError(RuntimeError):
@@ -73,6 +74,11 @@ def lib() -> ctypes.CDLL:
         L.attn_timing_enable.restype = ctypes.c_int
         L.attn_timing_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]
         L.attn_timing_read.restype = ctypes.c_int
+        L.attn_bwd_workspace_size.argtypes = [ctypes.POINTER(_Shape)]
+        L.attn_bwd_workspace_size.restype = sz
+        L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
+                               ctypes.c_float, ctypes.c_int, vp, ctypes.POINTER(_Shape), vp, sz]
+        L.attn_bwd.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -151,6 +157,60 @@ def attn_fwd(q, k, v, cu_seqlens, out, lse, causal: bool, scale: float, dtype: i
                         workspace.numel())
     if rc != 0:
         raise AttnError(rc, "attn_fwd")
+    return workspace
+
+
+def _doc_shape(q, cu_seqlens, max_seqlen, num_seqs) -> Shape:
+    T, H, d = q.shape
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+            raise ValueError("cu_seqlens must be an int32 CUDA tensor")
+        ns = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens (no host sync is done)")
+    else:
+        ns = num_seqs if num_seqs is not None else 1
+        if max_seqlen is None:
+            max_seqlen = T // max(ns, 1)
+    return Shape(T, ns, H, d, int(max_seqlen))
+
+
+def bwd_workspace_size(shape: Shape) -> int:
+    s = shape.c()
+    return int(lib().attn_bwd_workspace_size(ctypes.byref(s)))
+
+
+def make_bwd_workspace(shape: Shape, device=None) -> torch.Tensor:
+    n = bwd_workspace_size(shape)
+    if n == 0:
+        raise AttnError(1, "attn_bwd_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def attn_bwd(q, k, v, out, dout, lse, cu_seqlens, dq, dk, dv, causal: bool, scale: float,
+             stream=None, workspace=None, max_seqlen: int | None = None,
+             num_seqs: int | None = None):
+    """Gradients of the forward through the C ABI (``attn_bwd``): q, k, v,
+    out (the forward's output), dout: bf16 [T, H, d]; lse: fp32 [H, T] from
+    the forward; dq, dk, dv: bf16 [T, H, d], written.  Same document rules
+    as ``attn_fwd``.  Returns the workspace used (allocated if not given)."""
+    T, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("dq", dq),
+                    ("dk", dk), ("dv", dv)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (H, T):
+        raise ValueError("lse must be a contiguous fp32 tensor of shape [H, T]")
+    shape = _doc_shape(q, cu_seqlens, max_seqlen, num_seqs)
+    if workspace is None:
+        workspace = make_bwd_workspace(shape, q.device)
+    s = shape.c()
+    rc = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                        _ptr(cu_seqlens), _ptr(dq), _ptr(dk), _ptr(dv), int(bool(causal)),
+                        float(scale), ATTN_BF16, _stream_handle(stream, q.device),
+                        ctypes.byref(s), _ptr(workspace), workspace.numel())
+    if rc != 0:
+        raise AttnError(rc, "attn_bwd")
     return workspace
 
 

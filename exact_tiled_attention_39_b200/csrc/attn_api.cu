@@ -424,3 +424,159 @@ extern "C" attn_status_t attn_fwd_noalloc(const void* q, const void* k, const vo
   return attn_fwd(q, k, v, cu_seqlens, out, lse, causal, scale, ATTN_BF16, stream, shape,
                   scratch, kNoAllocScratchBytes);
 }
+
+// ===========================================================================
+// Backward (bf16): attn_bwd_workspace_size, attn_bwd.  The forward's sources
+// end above this line.
+// ===========================================================================
+#include "attn_bwd_sm100.cuh"
+
+namespace attn {
+namespace {
+
+struct BwdWsLayout {
+  size_t sorted_off, unsorted_off, delta_off, dq_off, total;
+  int64_t max_entries;
+};
+
+BwdWsLayout bwd_ws_layout(const attn_shape_t& s) {
+  BwdWsLayout w{};
+  w.max_entries = max_work_entries(s.total_tokens, s.num_seqs);
+  w.sorted_off = kWsListOffset;
+  w.unsorted_off = align_up(w.sorted_off + 16 * static_cast<size_t>(w.max_entries), kWsAlign);
+  w.delta_off = align_up(w.unsorted_off + 16 * static_cast<size_t>(w.max_entries), kWsAlign);
+  const size_t rows = static_cast<size_t>(s.total_tokens) * s.num_heads;
+  w.dq_off = align_up(w.delta_off + 4 * rows, kWsAlign);
+  w.total = align_up(w.dq_off + 4 * rows * s.head_dim, kWsAlign);
+  return w;
+}
+
+bool g_bwd_ready[kMaxDevices] = {};
+
+attn_status_t bwd_kernel_attributes(int dev) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_bwd_ready[dev]) return ATTN_OK;
+  if (cudaFuncSetAttribute(attn_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           BwdLayout<64>::kBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(attn_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           BwdLayout<128>::kBytes) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  g_bwd_ready[dev] = true;
+  return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace attn
+
+extern "C" {
+
+size_t attn_bwd_workspace_size(const attn_shape_t* shape) {
+  if (check_shape(shape) != ATTN_OK) return 0;
+  return bwd_ws_layout(*shape).total;
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, const int32_t* cu_seqlens, void* dq,
+                       void* dk, void* dv, int causal, float scale, attn_dtype_t dtype,
+                       void* stream, const attn_shape_t* shape, void* workspace,
+                       size_t workspace_bytes) {
+  const attn_status_t st = check_shape(shape);
+  if (st != ATTN_OK) return st;
+  if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  const attn_shape_t s = *shape;
+  if (cu_seqlens == nullptr &&
+      static_cast<int64_t>(s.num_seqs) * s.max_seqlen != static_cast<int64_t>(s.total_tokens))
+    return ATTN_ERR_INVALID_ARG;
+  if (s.total_tokens == 0) return ATTN_OK;
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  const void* ptrs[9] = {q, k, v, out, dout, lse, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return ATTN_ERR_ALIGNMENT;
+  const BwdWsLayout wl = bwd_ws_layout(s);
+  if (workspace == nullptr || workspace_bytes < wl.total) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
+
+  int dev = 0;
+  DeviceInfo info;
+  if (device_info(&dev, &info) != ATTN_OK) return ATTN_ERR_CUDA;
+  if (bwd_kernel_attributes(dev) != ATTN_OK) return ATTN_ERR_CUDA;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* header = reinterpret_cast<int32_t*>(ws);
+  float* delta = reinterpret_cast<float*>(ws + wl.delta_off);
+  float* dq_acc = reinterpret_cast<float*>(ws + wl.dq_off);
+
+  // 1. schedule: one entry per 128-token tile of each document, heaviest
+  //    first (validates cu_seqlens)
+  const int64_t cap = sort_capacity_for(wl.max_entries);
+  build_schedule_kernel<<<1, kScheduleThreads, static_cast<size_t>(cap) * 8, strm>>>(
+      cu_seqlens, s.num_seqs, s.total_tokens, s.max_seqlen, s.max_seqlen, causal, 1, header,
+      reinterpret_cast<int4*>(ws + wl.sorted_off), reinterpret_cast<int4*>(ws + wl.unsorted_off),
+      static_cast<int>(cap));
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+  // 2. D = rowsum(dO * O), dQ accumulator cleared
+  const long long rows = static_cast<long long>(s.total_tokens) * s.num_heads;
+  const long long prep_threads = rows * (s.head_dim / 8);
+  const long long prep_grid = (prep_threads + 255) / 256;
+  if (prep_grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  attn_bwd_prep_kernel<<<static_cast<unsigned>(prep_grid), 256, 0, strm>>>(
+      static_cast<const uint4*>(out), static_cast<const uint4*>(dout), delta,
+      reinterpret_cast<float4*>(dq_acc), rows, s.head_dim, s.num_heads, s.total_tokens);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+  // 3. dK, dV and the dQ partial sums, one key tile per unit
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_qkv_map(&tq, q, s.total_tokens, s.num_heads, s.head_dim, 2) ||
+      !encode_qkv_map(&tk, k, s.total_tokens, s.num_heads, s.head_dim, 2) ||
+      !encode_qkv_map(&tv, v, s.total_tokens, s.num_heads, s.head_dim, 2) ||
+      !encode_qkv_map(&tdo, dout, s.total_tokens, s.num_heads, s.head_dim, 2))
+    return ATTN_ERR_CUDA;
+  BwdParams bp;
+  bp.lse = lse;
+  bp.delta = delta;
+  bp.dq_acc = dq_acc;
+  bp.dk = dk;
+  bp.dv = dv;
+  bp.ws_header = header;
+  bp.work = reinterpret_cast<const int4*>(ws + wl.sorted_off);
+  bp.err = header + kWsErrorOffset / 4;
+  bp.total_tokens = s.total_tokens;
+  bp.num_heads = s.num_heads;
+  // Q and dO of a head are what every key tile of it reads again.
+  bp.head_groups = head_group_count(s.total_tokens, s.num_heads, s.head_dim, 4);
+  bp.causal = causal;
+  bp.scale = scale;
+  bp.scale_log2 = scale * 1.4426950408889634f;
+  bp.timeout_ns = kWaitTimeoutNs;
+  const int64_t max_units = wl.max_entries * s.num_heads;
+  const int grid = static_cast<int>(max_units < info.num_sms ? max_units : info.num_sms);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kBwdThreads);
+  cfg.stream = strm;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (s.head_dim == 128) {
+    cfg.dynamicSmemBytes = BwdLayout<128>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_bwd_kernel<128>, tq, tk, tv, tdo, bp);
+  } else {
+    cfg.dynamicSmemBytes = BwdLayout<64>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_bwd_kernel<64>, tq, tk, tv, tdo, bp);
+  }
+  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+  // 4. dQ = scale * accumulator in bf16
+  const long long n4 = rows * s.head_dim / 4;
+  attn_bwd_dq_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, strm>>>(
+      bp.err, reinterpret_cast<const float4*>(dq_acc), static_cast<uint2*>(dq), n4, scale);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

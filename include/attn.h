@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define ATTN_ABI_VERSION 2
+#define ATTN_ABI_VERSION 3
 
 typedef enum {
   ATTN_BF16 = 0,  /* bf16 operands, bf16 tensor-core products, fp32 softmax   */
@@ -171,6 +171,36 @@ attn_status_t attn_get_device_error(const void* workspace, void* stream,
  * events fail. */
 attn_status_t attn_timing_enable(int32_t enable);
 attn_status_t attn_timing_read(float* attention_ms, float* prepass_ms);
+
+/* Bytes of device workspace attn_bwd needs for this shape (0 for an invalid
+ * shape): the error word and work lists as for attn_fwd, then D (fp32
+ * [H, T]) and the fp32 dQ accumulator ([T, H, d]). */
+size_t attn_bwd_workspace_size(const attn_shape_t* shape);
+
+/* Exact attention backward: the gradients of attn_fwd's output with respect
+ * to q, k and v, given the upstream gradient dout.  The pages print no
+ * backward formulas (FLAMIA, section "Performans Sonuçları", measures forward
+ * and backward together); these are the derivatives of the definition
+ * above, per document and head, with P recomputed from the saved lse:
+ *     P = exp(scale S - lse),  dV = P^T dO,  dP = dO V^T,
+ *     D_i = dO_i . O_i,  dS = P * (dP - D),
+ *     dQ = scale dS K,  dK = scale dS^T Q.
+ * q, k, v, out, dout: bf16 [T, H, d] (out and lse as attn_fwd wrote them for
+ * the same q, k, v, cu_seqlens, causal and scale); lse: fp32 [H, T];
+ * dq, dk, dv: bf16 [T, H, d], written.  Same cu_seqlens, shape and causal
+ * rules as attn_fwd; dtype must be ATTN_BF16 (ATTN_ERR_UNSUPPORTED
+ * otherwise); head dim 64 or 128.  Launches the schedule-build kernel, a
+ * kernel computing D and clearing the accumulator, the backward kernel (one
+ * 128-key tile of a document and head per work unit; dK and dV accumulate
+ * on chip, dQ through fp32 vector reductions, so dq is not bit-reproducible
+ * across calls) and the kernel that scales and rounds dQ.  Device faults
+ * (bad cu_seqlens, a wait running out) are recorded in the workspace's error
+ * word as for attn_fwd and leave dq unwritten. */
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, const int32_t* cu_seqlens, void* dq,
+                       void* dk, void* dv, int causal, float scale, attn_dtype_t dtype,
+                       void* stream, const attn_shape_t* shape, void* workspace,
+                       size_t workspace_bytes);
 
 /* Static, human-readable name of a status code. */
 const char* attn_status_string(attn_status_t status);

@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_version_and_strings(L):
-    assert L.attn_abi_version() == 2
+    assert L.attn_abi_version() == 3
     assert A.status_string(0) == "ATTN_OK"
     assert A.status_string(5) == "ATTN_ERR_BAD_SEQLENS"
     assert A.status_string(6) == "ATTN_ERR_TIMEOUT"
@@ -96,3 +96,45 @@ def test_timing_read_without_a_timed_call(L):
     assert L.attn_timing_read(ctypes.byref(a), ctypes.byref(b)) == 1
     assert L.attn_timing_read(None, None) == 1
     A.attn_timing_enable(False)
+
+
+def _bwd(L, shape, n_null=None, misalign=None, ws=16, ws_bytes=1 << 30, scale=0.125, causal=1,
+         dtype=0):
+    s = shape.c() if shape is not None else None
+    ptrs = [16] * 10      # q k v out dout lse cu dq dk dv (cu at index 6: NULL = dense)
+    ptrs[6] = 0
+    if n_null is not None:
+        ptrs[n_null] = 0
+    if misalign is not None:
+        ptrs[misalign] = 24
+    args = [ctypes.c_void_p(p) if p else None for p in ptrs]
+    return L.attn_bwd(*args, causal, scale, dtype, None,
+                      ctypes.byref(s) if s is not None else None,
+                      ctypes.c_void_p(ws) if ws else None, ws_bytes)
+
+
+def test_bwd_workspace_size(L):
+    s = A.Shape(16384, 7, 32, 128, 4096)
+    n = A.bwd_workspace_size(s)
+    max_entries = 16384 // 128 + 7 + 1
+    # lists, D (fp32 [H, T]) and the fp32 dQ accumulator
+    assert n >= 256 + 2 * 16 * max_entries + 4 * 16384 * 32 + 4 * 16384 * 32 * 128
+    assert A.bwd_workspace_size(A.Shape(16, 1, 1, 96, 16)) == 0
+    assert A.bwd_workspace_size(A.Shape(-1, 1, 1, 64, 16)) == 0
+
+
+def test_bwd_host_checks_return_before_launch(L):
+    ok = A.Shape(256, 1, 2, 64, 256)
+    assert _bwd(L, None) == 1
+    assert _bwd(L, A.Shape(256, 1, 2, 96, 256)) == 2            # d unsupported
+    assert _bwd(L, ok, dtype=1) == 2                            # MXFP8 backward: not built
+    assert _bwd(L, ok, scale=-1.0) == 1
+    assert _bwd(L, ok, causal=3) == 1
+    assert _bwd(L, A.Shape(256, 2, 2, 64, 100)) == 1            # dense: T != B*N
+    for i in (0, 3, 4, 5, 7, 9):
+        assert _bwd(L, ok, n_null=i) == 1
+    for i in (1, 4, 5, 8):
+        assert _bwd(L, ok, misalign=i) == 3
+    assert _bwd(L, ok, ws=0) == 4
+    assert _bwd(L, ok, ws_bytes=64) == 4
+    assert _bwd(L, A.Shape(0, 0, 2, 64, 0)) == 0                # T == 0: no-op
