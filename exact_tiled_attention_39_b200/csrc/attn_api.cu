@@ -453,6 +453,22 @@ BwdWsLayout bwd_ws_layout(const attn_shape_t& s) {
 
 bool g_bwd_ready[kMaxDevices] = {};
 
+// 3-D map over the fp32 dQ accumulator [T, H, d] for the kernel's reduce-add
+// copies: box = 32 fp32 of head dim (128 bytes, the swizzle span) x 1 head x
+// 32 tokens, 128-byte swizzle.
+bool encode_dq_map(CUtensorMap* m, void* base, int T, int H, int d) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(H) * d * 4};
+  const cuuint32_t box[3] = {32, 1, 32};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 attn_status_t bwd_kernel_attributes(int dev) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (g_bwd_ready[dev]) return ATTN_OK;
@@ -528,11 +544,12 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
   // 3. dK, dV and the dQ partial sums, one key tile per unit
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   if (!encode_qkv_map(&tq, q, s.total_tokens, s.num_heads, s.head_dim, 2) ||
       !encode_qkv_map(&tk, k, s.total_tokens, s.num_heads, s.head_dim, 2) ||
       !encode_qkv_map(&tv, v, s.total_tokens, s.num_heads, s.head_dim, 2) ||
-      !encode_qkv_map(&tdo, dout, s.total_tokens, s.num_heads, s.head_dim, 2))
+      !encode_qkv_map(&tdo, dout, s.total_tokens, s.num_heads, s.head_dim, 2) ||
+      !encode_dq_map(&tdq, dq_acc, s.total_tokens, s.num_heads, s.head_dim))
     return ATTN_ERR_CUDA;
   BwdParams bp;
   bp.lse = lse;
@@ -565,10 +582,10 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   cudaError_t e;
   if (s.head_dim == 128) {
     cfg.dynamicSmemBytes = BwdLayout<128>::kBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_bwd_kernel<128>, tq, tk, tv, tdo, bp);
+    e = cudaLaunchKernelEx(&cfg, attn_bwd_kernel<128>, tq, tk, tv, tdo, tdq, bp);
   } else {
     cfg.dynamicSmemBytes = BwdLayout<64>::kBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_bwd_kernel<64>, tq, tk, tv, tdo, bp);
+    e = cudaLaunchKernelEx(&cfg, attn_bwd_kernel<64>, tq, tk, tv, tdo, tdq, bp);
   }
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 

@@ -23,8 +23,9 @@
 // A work unit is one 128-key tile K_j, V_j of one document and head.  The
 // CTA keeps dK_j and dV_j in TMEM while it walks the query tiles that see
 // K_j (causal: from the diagonal tile on).  dQ_i gets one partial product
-// per (i, j); it is added in fp32 to a device accumulator with vector
-// reductions, and a last small kernel scales and rounds it.
+// per (i, j); it is added in fp32 to a device accumulator by TMA tensor
+// reductions (staged in shared memory, 32 rows x 32 columns per copy), and a
+// last small kernel scales and rounds it.
 //
 // Orientation: TMEM lane = key.  S^T = K_j Q_i^T and dP^T = V_j dO_i^T give
 // each thread one key row of 128 query columns; P^T and dS^T go back over
@@ -34,8 +35,10 @@
 //
 //   warps 0..3    compute: P^T from S^T, lse and the masks; dS^T from dP^T
 //                 and D (one key row per thread).
-//   warps 4..7    dQ_i read-out and fp32 reductions into the accumulator;
-//                 at the end of a unit the dK_j, dV_j epilogue.
+//   warps 4..7    dQ_i read-out: TMEM -> registers -> shared memory (the dS
+//                 buffer, free once dQ_i's product has read it) -> TMA
+//                 reduce-add into the accumulator; at the end of a unit the
+//                 dK_j, dV_j epilogue.
 //   warp 8        producer: claims units; TMA loads of K_j, V_j and of Q_i,
 //                 dO_i into a two-stage ring, with the tile's lse and D rows.
 //   warp 9        MMA issuer (one thread).
@@ -44,6 +47,11 @@
 // TMEM (512 columns): S^T / P^T at 0; dP^T / dS^T at 128, where dQ_i lands
 // once dK's product has read dS^T (the tensor pipe runs products in issue
 // order); dV at 256, dK at 256 + D.
+//
+// A 128-row query tile may run past its document's end into the next
+// document.  Those rows have P = 0, hence dS = 0 and a dQ_i row of exact
+// zeros, so the reduction copies cover whole 32-row boxes: they add +-0 to
+// the next document's rows (rows past the tensor's end are clipped by TMA).
 #pragma once
 #include <cuda.h>
 
@@ -88,8 +96,11 @@ struct BwdLayout {
   static constexpr int kStageBytes = 2 * kTileBytes;          // Q_i, then dO_i
   static constexpr int kRingOff = 2 * kTileBytes;
   // dS (bf16, 128 queries x 128 keys), MN-major: row = key, 64 queries per
-  // 128-byte chunk row, two chunks of 16 KB.
+  // 128-byte chunk row, two chunks of 16 KB.  Between dQ_i's product and
+  // the next dS it is the dQ staging area: per read-out warp two 4 KB
+  // buffers of 32 rows x 32 fp32 in the 128-byte swizzle.
   static constexpr int kDsOff = kRingOff + kStages * kStageBytes;
+  static constexpr int kStageBufBytes = 32 * 128;
   static constexpr int kDsBytes = 2 * kChunkBytes;
   static constexpr int kVecOff = kDsOff + kDsBytes;           // float [stage][lse2, D][128]
   static constexpr int kBarOff = kVecOff + kStages * 2 * 128 * 4;
@@ -104,7 +115,8 @@ struct BwdLayout {
   static constexpr int kDQEmpty = kDQFull + 1;
   static constexpr int kDKVFull = kDQEmpty + 1;
   static constexpr int kDKVEmpty = kDKVFull + 1;
-  static constexpr int kDrain = kDKVEmpty + 1;
+  static constexpr int kDsFree = kDKVEmpty + 1;              // staging read by the reductions
+  static constexpr int kDrain = kDsFree + 1;
   static constexpr int kUnitFull = kDrain + 1;                // + slot
   static constexpr int kUnitEmpty = kUnitFull + kUnitSlots;   // + slot
   static constexpr int kNumBars = kUnitEmpty + kUnitSlots;
@@ -112,12 +124,35 @@ struct BwdLayout {
   static constexpr int kUnitOff = kMiscOff + 16;              // int4 [kUnitSlots]
   static constexpr int kBytes = kUnitOff + 16 * kUnitSlots;
   static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
+  static_assert(4 * 2 * kStageBufBytes <= kDsBytes, "dQ staging must fit the dS buffer");
   static constexpr uint32_t kTmemS = 0;
   static constexpr uint32_t kTmemDP = 128;
   static constexpr uint32_t kTmemDV = 256;
   static constexpr uint32_t kTmemDK = 256 + D;
   static constexpr uint32_t kTmemCols = 512;
 };
+
+// TMA tensor reduce-add of a shared-memory box into global memory (element
+// type and box from the tensor map), tracked by the issuing thread's bulk
+// async-group.
+__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int32_t c0,
+                                                  int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 
 // D = rowsum(dO * O) per (token, head) into [H, T], and the dQ accumulator
 // row cleared.  d / 8 threads per row, 8 elements each.
@@ -170,7 +205,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                const BwdParams p) {
+                const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using Lay = BwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = ptx::smem_addr(smem);
@@ -202,6 +237,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     ptx::mbar_init(bar(Lay::kDQEmpty), 4);
     ptx::mbar_init(bar(Lay::kDKVFull), 1);
     ptx::mbar_init(bar(Lay::kDKVEmpty), 4);
+    ptx::mbar_init(bar(Lay::kDsFree), 4);
     ptx::mbar_init(bar(Lay::kDrain), 1);
     for (int i = 0; i < kUnitSlots; ++i) {
       ptx::mbar_init(bar(Lay::kUnitFull + i), 1);
@@ -215,6 +251,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     ptx::prefetch_tmap(&tm_k);
     ptx::prefetch_tmap(&tm_v);
     ptx::prefetch_tmap(&tm_do);
+    ptx::prefetch_tmap(&tm_dq);
   }
   if (warp == kWarpMma) {
     ptx::tmem_alloc(ptx::smem_addr(tmem_holder), Lay::kTmemCols);
@@ -310,6 +347,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // dP^T in TMEM and as a row of the MN-major dS tile in shared memory
         if (!(ok = wait_warp(bar(Lay::kDPFull), q_cnt & 1, ctl))) break;
         ptx::tc_fence_after();
+        // the dS buffer: the previous step's dQ staging must have been read
+        if (q_cnt > 0 && !(ok = wait_warp(bar(Lay::kDsFree), (q_cnt - 1) & 1, ctl))) break;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t dp[32];
@@ -350,6 +389,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t stage_base = sbase + Lay::kDsOff + wq * 2 * Lay::kStageBufBytes;
     uint32_t q_cnt = 0, u_cnt = 0;
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
@@ -372,16 +412,37 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(Lay::kDQEmpty));
-        const int row = qb * kBlockM + r;
-        if (row < uw.y) {
-          float4* dst = reinterpret_cast<float4*>(
-              p.dq_acc + (static_cast<long long>(uw.x + row) * H + uw.w) * D);
+        // 32 columns per copy: this warp's 32 rows in a 4 KB buffer (row =
+        // lane, 16-byte unit u at u ^ (lane % 8)), two buffers in turn
+        const int qrow0 = uw.x + qb * kBlockM + 32 * wq;
+        // (a warp whose 32 rows all lie past the document end has only zeros)
+        const bool any_row = qb * kBlockM + 32 * wq < uw.y;
 #pragma unroll
-          for (int a = 0; a < D / 4; ++a)
-            atomicAdd(dst + a, make_float4(__uint_as_float(acc[4 * a]), __uint_as_float(acc[4 * a + 1]),
-                                           __uint_as_float(acc[4 * a + 2]),
-                                           __uint_as_float(acc[4 * a + 3])));
+        for (int c = 0; c < D / 32; ++c) {
+          if (!any_row) break;
+          if (c >= 2) {
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+          }
+          const uint32_t buf = stage_base + (c & 1) * Lay::kStageBufBytes;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t addr = buf + lane * 128 + ((u ^ (lane & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                         "r"(acc[32 * c + 4 * u]), "r"(acc[32 * c + 4 * u + 1]),
+                         "r"(acc[32 * c + 4 * u + 2]), "r"(acc[32 * c + 4 * u + 3])
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_3d(&tm_dq, buf, 32 * c, uw.w, qrow0);
+            bulk_commit_group();
+          }
         }
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(Lay::kDsFree));
       }
       if (!ok) break;
       // dK_j, dV_j of the unit (key rows)
