@@ -33,20 +33,25 @@
 // TMEM.  dQ_i = dS K_j reads dS from shared memory, stored MN-major (a key
 // row of dS^T is a column of dS).
 //
-//   warps 0..3    compute: P^T from S^T, lse and the masks; dS^T from dP^T
-//                 and D (one key row per thread).
-//   warps 4..7    dQ_i read-out: TMEM -> registers -> shared memory (the dS
-//                 buffer, free once dQ_i's product has read it) -> TMA
-//                 reduce-add into the accumulator; at the end of a unit the
-//                 dK_j, dV_j epilogue.
-//   warp 8        producer: claims units; TMA loads of K_j, V_j and of Q_i,
-//                 dO_i into a two-stage ring, with the tile's lse and D rows.
-//   warp 9        MMA issuer (one thread).
-//   warps 10..11  idle.
+//   warps 0..7    compute, two warpgroups on the same key rows: warpgroup g
+//                 takes query columns [64 g, 64 g + 64).  P^T from S^T, lse
+//                 and the masks; dS^T from dP^T and D.  Each half writes its
+//                 bf16 values over the first 32 columns of its own 64, so
+//                 neither overwrites what the other has still to read.
+//   warps 8..11   dQ_i read-out (176 registers): TMEM -> registers -> shared
+//                 memory (the dS buffer, free once dQ_i's product has read
+//                 it) -> TMA reduce-add into the accumulator; at the end of a
+//                 unit the dK_j, dV_j epilogue.
+//   warp 12       producer (80 registers): claims units; TMA loads of K_j,
+//                 V_j and of Q_i, dO_i into a two-stage ring, with the tile's
+//                 lse and D rows.
+//   warp 13       MMA issuer (one thread).
+//   warps 14..15  idle.
 //
 // TMEM (512 columns): S^T / P^T at 0; dP^T / dS^T at 128, where dQ_i lands
 // once dK's product has read dS^T (the tensor pipe runs products in issue
-// order); dV at 256, dK at 256 + D.
+// order); dV at 256, dK at 256 + D.  The bf16 P^T and dS^T of query columns
+// [64 g, 64 g + 64) sit in TMEM columns [64 g, 64 g + 32) of their block.
 //
 // A 128-row query tile may run past its document's end into the next
 // document.  Those rows have P = 0, hence dS = 0 and a dQ_i row of exact
@@ -81,8 +86,15 @@ struct BwdParams {
   unsigned long long timeout_ns;
 };
 
-constexpr int kBwdThreads = 384;
-constexpr int kBwdUnitConsumers = 1 + 4 + 4;   // MMA thread, compute warps, read-out warps
+constexpr int kBwdThreads = 512;
+constexpr int kBwdComputeWarps = 8;
+constexpr int kBwdUnitConsumers = 1 + kBwdComputeWarps + 4;   // MMA thread, compute, read-out warps
+// Registers per thread at launch: 65536 / 512 = 128.  The compute
+// warpgroups keep 128; the read-out warpgroup takes what the producer / MMA
+// warpgroup gives up.
+constexpr uint32_t kBwdRegsCompute = 128, kBwdRegsReadout = 176, kBwdRegsOther = 80;
+static_assert(2 * kBwdRegsCompute + kBwdRegsReadout + kBwdRegsOther == 4 * 128,
+              "register split must use exactly the registers the CTA is launched with");
 
 template <int D>
 struct BwdLayout {
@@ -221,18 +233,18 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   float* vecs = reinterpret_cast<float*>(smem + Lay::kVecOff);
   int4* unit_ring = reinterpret_cast<int4*>(smem + Lay::kUnitOff);
 
-  constexpr int kWarpTma = 8, kWarpMma = 9;
+  constexpr int kWarpTma = 12, kWarpMma = 13;
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(Lay::kKVFull), 1);
     ptx::mbar_init(bar(Lay::kKVEmpty), 1);
     for (int s = 0; s < Lay::kStages; ++s) {
       ptx::mbar_init(bar(Lay::kQFull + s), 1);
-      ptx::mbar_init(bar(Lay::kQEmpty + s), 1 + 4);   // MMA commit + compute warps (lse, D)
+      ptx::mbar_init(bar(Lay::kQEmpty + s), 1 + kBwdComputeWarps);   // MMA + compute (lse, D)
     }
     ptx::mbar_init(bar(Lay::kSFull), 1);
-    ptx::mbar_init(bar(Lay::kPFull), 4);
+    ptx::mbar_init(bar(Lay::kPFull), kBwdComputeWarps);
     ptx::mbar_init(bar(Lay::kDPFull), 1);
-    ptx::mbar_init(bar(Lay::kDSFull), 4);
+    ptx::mbar_init(bar(Lay::kDSFull), kBwdComputeWarps);
     ptx::mbar_init(bar(Lay::kDQFull), 1);
     ptx::mbar_init(bar(Lay::kDQEmpty), 4);
     ptx::mbar_init(bar(Lay::kDKVFull), 1);
@@ -286,14 +298,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     return n_tiles - qb0;
   };
 
-  if (warp < 4) {
+  if (warp < 8) {
     // ------------------------------------------------------------ compute
-    const int r = warp * 32 + lane;                // key row within the tile
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_off + Lay::kTmemS;
-    const uint32_t t_dp = tmem + lane_off + Lay::kTmemDP;
+    const int g = warp >> 2;                       // query-column half
+    const int r = (warp & 3) * 32 + lane;          // key row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + Lay::kTmemS + 64 * g;
+    const uint32_t t_dp = tmem + lane_off + Lay::kTmemDP + 64 * g;
     const float c = p.scale_log2;
-    uint8_t* const ds_row = smem + Lay::kDsOff + r * 128;
+    uint8_t* const ds_row = smem + Lay::kDsOff + g * Lay::kChunkBytes + r * 128;
     uint32_t q_cnt = 0;                            // query steps so far (all units)
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
@@ -307,33 +320,31 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int qb = qb0 + ii;
         const uint32_t s = q_cnt % Lay::kStages;
         if (!(ok = wait_warp(bar(Lay::kQFull + s), (q_cnt / Lay::kStages) & 1, ctl))) break;
-        const float* lse2 = vecs + (s * 2) * 128;
-        const float* dd = vecs + (s * 2 + 1) * 128;
-        // visible query columns: q < q_end, and q >= r on the diagonal tile
-        const int q_end = key_ok ? min(uw.y - qb * kBlockM, kBlockM) : 0;
-        const int q_begin = (causal && qb == kb) ? r : 0;
+        const float* lse2 = vecs + (s * 2) * 128 + 64 * g;
+        const float* dd = vecs + (s * 2 + 1) * 128 + 64 * g;
+        // visible query columns q (relative to this half): 64 g + q < q_end,
+        // and 64 g + q >= r on the diagonal tile
+        const int q_end = (key_ok ? min(uw.y - qb * kBlockM, kBlockM) : 0) - 64 * g;
+        const int q_begin = ((causal && qb == kb) ? r : 0) - 64 * g;
         if (!(ok = wait_warp(bar(Lay::kSFull), q_cnt & 1, ctl))) break;
         ptx::tc_fence_after();
-        uint32_t pk[64];   // P^T row as bf16 pairs
+        uint32_t pk[32];   // this half of the P^T row as bf16 pairs
         {
           uint32_t sa[64];
+          ptx::tmem_ld_x64(t_s, sa);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            ptx::tmem_ld_x64(t_s + 64 * h, sa);
-#pragma unroll
-            for (int a = 0; a < 32; ++a) {
-              const int q = 64 * h + 2 * a;
-              const float2 l2 = *reinterpret_cast<const float2*>(lse2 + q);
-              float p0 = ptx::ex2_approx(__uint_as_float(sa[2 * a]) * c - l2.x);
-              float p1 = ptx::ex2_approx(__uint_as_float(sa[2 * a + 1]) * c - l2.y);
-              if (q < q_begin || q >= q_end) p0 = 0.f;
-              if (q + 1 < q_begin || q + 1 >= q_end) p1 = 0.f;
-              pk[32 * h + a] = ptx::pack_bf16x2(p0, p1);
-            }
+          for (int a = 0; a < 32; ++a) {
+            const int q = 2 * a;
+            const float2 l2 = *reinterpret_cast<const float2*>(lse2 + q);
+            float p0 = ptx::ex2_approx(__uint_as_float(sa[2 * a]) * c - l2.x);
+            float p1 = ptx::ex2_approx(__uint_as_float(sa[2 * a + 1]) * c - l2.y);
+            if (q < q_begin || q >= q_end) p0 = 0.f;
+            if (q + 1 < q_begin || q + 1 >= q_end) p1 = 0.f;
+            pk[a] = ptx::pack_bf16x2(p0, p1);
           }
         }
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           uint32_t w[16];
 #pragma unroll
           for (int a = 0; a < 16; ++a) w[a] = pk[16 * ch + a];
@@ -344,13 +355,14 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(Lay::kPFull));
         // dS^T = P^T * (dP^T - D), 32 query columns at a time, written over
-        // dP^T in TMEM and as a row of the MN-major dS tile in shared memory
+        // this half's dP^T in TMEM and as chunk g of the key's row of the
+        // MN-major dS tile in shared memory
         if (!(ok = wait_warp(bar(Lay::kDPFull), q_cnt & 1, ctl))) break;
         ptx::tc_fence_after();
         // the dS buffer: the previous step's dQ staging must have been read
         if (q_cnt > 0 && !(ok = wait_warp(bar(Lay::kDsFree), (q_cnt - 1) & 1, ctl))) break;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           uint32_t dp[32];
           ptx::tmem_ld_x32(t_dp + 32 * ch, dp);
           uint32_t ds[16];
@@ -363,14 +375,14 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ds[a] = ptx::pack_bf16x2(p0 * (__uint_as_float(dp[2 * a]) - d2.x),
                                      p1 * (__uint_as_float(dp[2 * a + 1]) - d2.y));
           }
+          // columns 16 ch .. 16 ch + 15 of this half: dP^T values already read
           ptx::tmem_st_x16(t_dp + 16 * ch, ds);
-          // queries 32 ch .. 32 ch + 31: chunk ch / 2, 16-byte units
-          // 4 (ch % 2) .. 4 (ch % 2) + 3 of the row, swizzled by r % 8
+          // queries 32 ch .. 32 ch + 31 of the half: 16-byte units
+          // 4 ch .. 4 ch + 3 of the chunk row, swizzled by r % 8
 #pragma unroll
           for (int uu = 0; uu < 4; ++uu) {
-            const int u = 4 * (ch & 1) + uu;
-            *reinterpret_cast<uint4*>(ds_row + (ch >> 1) * Lay::kChunkBytes +
-                                      ((u ^ (r & 7)) << 4)) =
+            const int u = 4 * ch + uu;
+            *reinterpret_cast<uint4*>(ds_row + ((u ^ (r & 7)) << 4)) =
                 make_uint4(ds[4 * uu], ds[4 * uu + 1], ds[4 * uu + 2], ds[4 * uu + 3]);
           }
         }
@@ -384,8 +396,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------------------ dQ read-out, dK / dV epilogue
+    ptx::regs_increase<kBwdRegsReadout>();
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -480,7 +493,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
     }
-  } else if (warp == kWarpTma) {
+  } else {
+    ptx::regs_decrease<kBwdRegsOther>();
+  }
+  if (warp == kWarpTma) {
     // ------------------------------------------------------------ producer
     const int n_units = p.ws_header[kWsCountOffset / 4] * H;
     int* counter = const_cast<int*>(p.ws_header) + kWsUnitCounterOffset / 4;
@@ -645,7 +661,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlockM / 16; ++kk)
-          ptx::mma_f16_ts(tmem + Lay::kTmemDV, tmem + Lay::kTmemS + kk * 8,
+          ptx::mma_f16_ts(tmem + Lay::kTmemDV, tmem + Lay::kTmemS + kk * 8 + (kk >= 4 ? 32 : 0),
                           ptx::sdesc_join(do_lo + mn_lbo + kk * (2048 >> 4), kDescHi), kIdescG,
                           (ii > 0 || kk > 0) ? 1u : 0u);
         // dK += dS^T Q_i, then dQ_i = dS K_j over dS^T's columns
@@ -653,7 +669,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ptx::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlockM / 16; ++kk)
-          ptx::mma_f16_ts(tmem + Lay::kTmemDK, tmem + Lay::kTmemDP + kk * 8,
+          ptx::mma_f16_ts(tmem + Lay::kTmemDK, tmem + Lay::kTmemDP + kk * 8 + (kk >= 4 ? 32 : 0),
                           ptx::sdesc_join(q_lo + mn_lbo + kk * (2048 >> 4), kDescHi), kIdescG,
                           (ii > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
