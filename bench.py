@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload dense_causal|packed_causal|long_outlier|mxfp8_packed]
+                    [--pass fwd|bwd]
 
 One step = one ``attn_fwd`` call through the C ABI (the schedule-build
 kernel, the MXFP8 pre-pass for the MXFP8 workload, and the attention
@@ -13,6 +14,11 @@ cross-GPU exchange); the time is the max over ranks.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload and prints the same metric (rank 0 only).
+
+``--pass bwd`` times the backward instead (bf16 workloads): one step = one
+``attn_bwd`` call (schedule, D pre-pass, backward kernel, dQ conversion)
+with the forward's out and lse resident; FLOPs = 2.5 x the forward's (five
+products against two); the fp64 gradient oracle is the CPU baseline.
 """
 from __future__ import annotations
 
@@ -33,6 +39,7 @@ sys.path.insert(0, ROOT)
 from exact_tiled_attention_39_b200 import workloads  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s (causal, bf16 & MXFP8) and % of B200 dense tensor peak"
+METRIC_BWD = "attention bwd TFLOP/s (causal, bf16; 2.5 x forward FLOPs) and % of B200 dense tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -50,19 +57,19 @@ def load_peaks():
 BWD_SECTION_MARK = b"\n// " + b"=" * 75 + b"\n// Backward (bf16)"
 
 
-def kernel_sources_sha256() -> str:
-    """Hash of the CUDA sources the forward kernels are built and launched
-    from (names and bytes): every csrc file except the backward's, and
-    attn_api.cu up to its backward section."""
+def kernel_sources_sha256(part: str = "fwd") -> str:
+    """Hash of the CUDA sources (names and bytes) a kernel is built and
+    launched from.  "fwd": every csrc file except the backward's, and
+    attn_api.cu up to its backward section; "bwd": every csrc file."""
     import hashlib
     d = os.path.join(ROOT, "exact_tiled_attention_39_b200", "csrc")
     h = hashlib.sha256()
     for n in sorted(os.listdir(d)):
-        if n.endswith((".cu", ".cuh")) and not n.startswith("attn_bwd"):
+        if n.endswith((".cu", ".cuh")) and (part == "bwd" or not n.startswith("attn_bwd")):
             h.update(n.encode())
             with open(os.path.join(d, n), "rb") as f:
                 data = f.read()
-            if n == "attn_api.cu":
+            if n == "attn_api.cu" and part == "fwd":
                 cut = data.find(BWD_SECTION_MARK)
                 if cut >= 0:
                     data = data[:cut]
@@ -70,7 +77,7 @@ def kernel_sources_sha256() -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(workload: str, kernel: str):
+def recorded_traffic(workload: str, kernel: str, part: str = "fwd"):
     """DRAM bytes (read + write) per attention-kernel launch from the committed
     ncu summary of this kernel and workload, or None when there is none or it
     was taken on other kernel sources."""
@@ -84,7 +91,7 @@ def recorded_traffic(workload: str, kernel: str):
             for key in ("kernel_sources_sha256", "dram_bytes_per_launch"):
                 if line.startswith(key + ":"):
                     vals[key] = line.split(":", 1)[1].strip()
-    if vals.get("kernel_sources_sha256") != kernel_sources_sha256():
+    if vals.get("kernel_sources_sha256") != kernel_sources_sha256(part):
         return None
     try:
         return int(vals["dram_bytes_per_launch"])
@@ -387,6 +394,181 @@ def cpu_baseline(w, inp, budget_s=15.0):
                       f"{el:.1f} s"}
 
 
+def cpu_baseline_bwd(inp, dout, budget_s=15.0):
+    """The fp64 gradient oracle on the host cores on whole (document, head)
+    problems of the workload, largest documents first, within the budget."""
+    from oracle.attention_bwd import ref_attention_bwd
+
+    cores = len(os.sched_getaffinity(0))
+    torch.set_num_threads(cores)
+    lengths = inp["lengths"]
+    starts = np.concatenate([[0], np.cumsum(lengths)])
+    H, d = inp["q"].shape[1], inp["q"].shape[2]
+    problems = [(i, h) for i in np.argsort(lengths)[::-1] for h in range(H)]
+    done_flops, done = 0.0, 0
+    t_start = time.perf_counter()
+    for i, h in problems:
+        a, b = int(starts[i]), int(starts[i + 1])
+        x = [t[a:b, h:h + 1].double().numpy() for t in (inp["q"], inp["k"], inp["v"], dout)]
+        ref_attention_bwd(*x, [0, b - a], True, inp["scale"])
+        done_flops += 2.5 * workloads.flops([b - a], 1, d, True)
+        done += 1
+        if time.perf_counter() - t_start > budget_s:
+            break
+    el = time.perf_counter() - t_start
+    return {"value": round(done_flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{done} of {len(problems)} (document, head) problems, fp64 gradients, "
+                      f"{el:.1f} s"}
+
+
+def bench_ours_bwd(args):
+    from exact_tiled_attention_39_b200 import attn as A
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = init_group("nccl", dev)
+
+    w = workloads.get(args.workload)
+    if w.dtype != "bf16":
+        raise SystemExit("--pass bwd: the backward is built for bf16 workloads")
+    inp = workloads.make_inputs(w)
+    T, H, d = inp["q"].shape
+    causal = True
+    lengths = inp["lengths"]
+    max_seqlen = max(lengths)
+    flops = 2.5 * workloads.flops(lengths, H, d, causal)
+    g = torch.Generator().manual_seed(1000 + w.seed)
+    hdo = torch.randn((T, H, d), generator=g).to(torch.bfloat16)
+
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    do = hdo.to(dev)
+    cu = inp["cu_seqlens"].to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+    shape = A.Shape(T, len(lengths), H, d, max_seqlen)
+    A.attn_fwd(q, k, v, cu, out, lse, causal, inp["scale"], max_seqlen=max_seqlen)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = A.make_bwd_workspace(shape, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        A.attn_bwd(q, k, v, out, do, lse, cu, dq, dk, dv, causal, inp["scale"], stream=stream,
+                   workspace=ws, max_seqlen=max_seqlen)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert A.attn_get_device_error(ws) == 0, "device error during warm-up"
+
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    ms_total = max_over_ranks(pg, t0.elapsed_time(t1), dev)
+    ms_step = ms_total / args.steps
+    err = A.attn_get_device_error(ws)
+    value = aggregate_tflops(world, flops, ms_step)
+
+    # end to end: q, k, v, out, dout, lse, cu_seqlens in from pinned host
+    # memory, dq, dk, dv back
+    host_in = [inp["q"].pin_memory(), inp["k"].pin_memory(), inp["v"].pin_memory(),
+               out.cpu().pin_memory(), hdo.pin_memory(), lse.cpu().pin_memory(),
+               inp["cu_seqlens"].pin_memory()]
+    dev_in = [q, k, v, out, do, lse, cu]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+
+    def e2e_step():
+        for dst, src in zip(dev_in, host_in):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in zip(host_out, (dq, dk, dv)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(pg, s0.elapsed_time(s1) / e2e_steps, dev)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    peak_key = "bf16_tflops_sustained" if ms_total * 1e-3 > 1.0 else "bf16_tflops"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    line = {
+        "metric": METRIC_BWD,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, see workloads.py; dout seeded N(0,1))",
+        "config": {
+            "workload": f"{w.name} backward: {w.description}",
+            "tokens": T, "heads": H, "head_dim": d, "docs": len(lengths),
+            "causal": causal, "flops_per_step": flops,
+            "l2": f"inputs {6 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2; no flush",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "peak_source": f"{peak_source_name(peak_key, 0)} ({peak_src})",
+            "timed_unit": "whole attn_bwd call (4 kernels), device events over the timed steps",
+            "kernel": "attn_bwd_kernel",
+            "traffic": recorded_traffic(w.name, "attn_bwd_kernel", "bwd"),
+            "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
+        },
+        "e2e": {
+            "value": round(aggregate_tflops(world, flops, e2e_ms), 2),
+            "unit": "TFLOP/s",
+            "ms_per_step": round(e2e_ms, 3),
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+        },
+        "gpu_launches": args.steps * 4,
+        "clocks": clk.summary(),
+        "device_error": err,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_bwd(inp, hdo, budget_s=args.cpu_budget)
+    return line
+
+
 def bench_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -432,6 +614,7 @@ def main():
     ap.add_argument("--workload", default="dense_causal", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"])
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -441,7 +624,7 @@ def main():
         from exact_tiled_attention_39_b200 import build
         if dist_env()[1] == 0 or not os.path.exists(build.LIB):
             build.build()
-        line = bench_ours(args)
+        line = bench_ours_bwd(args) if args.which == "bwd" else bench_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)
 
