@@ -563,20 +563,23 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int ii = 0; ii < n; ++ii) {
         const int qb = qb0 + ii;
         const uint32_t s = q_it % Lay::kStages;
-        if (!(ok = wait_warp(bar(Lay::kQEmpty + s), ((q_it / Lay::kStages) & 1) ^ 1, ctl))) break;
-        // lse (in log2 units) and D of the tile's 128 query rows; rows past
-        // the document end get 0 (their columns are masked)
-        float* lv = vecs + (s * 2) * 128;
-        float* dv = vecs + (s * 2 + 1) * 128;
+        // lse (in log2 units) and D of the tile's 128 query rows, read before
+        // the stage is free so their latency overlaps the wait; rows past the
+        // document end get 0 (their columns are masked)
+        float lr[4], dr[4];
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
-          const int q = 4 * lane + a;
-          const int row = qb * kBlockM + q;
+          const int row = qb * kBlockM + 4 * lane + a;
           const bool valid = row < uw.y;
           const long long idx = static_cast<long long>(uw.w) * p.total_tokens + uw.x + row;
-          lv[q] = valid ? p.lse[idx] * kLog2e : 0.f;
-          dv[q] = valid ? p.delta[idx] : 0.f;
+          lr[a] = valid ? p.lse[idx] * kLog2e : 0.f;
+          dr[a] = valid ? p.delta[idx] : 0.f;
         }
+        if (!(ok = wait_warp(bar(Lay::kQEmpty + s), ((q_it / Lay::kStages) & 1) ^ 1, ctl))) break;
+        *reinterpret_cast<float4*>(vecs + (s * 2) * 128 + 4 * lane) =
+            make_float4(lr[0], lr[1], lr[2], lr[3]);
+        *reinterpret_cast<float4*>(vecs + (s * 2 + 1) * 128 + 4 * lane) =
+            make_float4(dr[0], dr[1], dr[2], dr[3]);
         __syncwarp();
         const uint32_t stage = sbase + Lay::kRingOff + s * Lay::kStageBytes;
         const int qrow0 = uw.x + qb * kBlockM;
@@ -672,6 +675,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           ptx::mma_f16_ts(tmem + Lay::kTmemDK, tmem + Lay::kTmemDP + kk * 8 + (kk >= 4 ? 32 : 0),
                           ptx::sdesc_join(q_lo + mn_lbo + kk * (2048 >> 4), kDescHi), kIdescG,
                           (ii > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(bar(Lay::kQEmpty + s));   // Q_i and dO_i: last read by dK's product
 #pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk)
           ptx::mma_f16_ss(tmem + Lay::kTmemDP,
@@ -679,7 +683,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                           ptx::sdesc_join(k_lo + mn_lbo + kk * (2048 >> 4), kDescHi), kIdescQ,
                           kk > 0 ? 1u : 0u);
         ptx::mma_commit(bar(Lay::kDQFull));
-        ptx::mma_commit(bar(Lay::kQEmpty + s));
       }
       if (!ok) break;
       ptx::mma_commit(bar(Lay::kDKVFull));
