@@ -1,6 +1,6 @@
 """Parity figures of the five configurations, one JSON line each (GPU).
 
-    python tests/parity_report.py
+    python tests/parity_report.py [--bwd-only]
 
 Runs every configuration through the C ABI and compares with the fp64 oracle
 the way the GPU tests do: the tiny config element by element (causal and
@@ -8,7 +8,10 @@ non-causal), the large ones on sampled rows (384 random rows plus every
 document's first, second, 128th, 129th, 256th, 257th and last row, random
 heads), MXFP8 against the oracle on the exactly dequantised inputs.  Prints
 max / mean absolute output error, max absolute lse error and the tolerance
-each is held to.  Test infrastructure, like the oracle it calls.
+each is held to.  Then the backward on the GPU tests' cases, every element of
+dq, dk, dv against the fp64 gradient oracle, errors relative to each
+gradient's largest magnitude.  Test infrastructure, like the oracle it
+calls.
 """
 from __future__ import annotations
 
@@ -26,6 +29,7 @@ sys.path.insert(0, HERE)
 from exact_tiled_attention_39_b200 import attn as A  # noqa: E402
 from exact_tiled_attention_39_b200 import workloads  # noqa: E402
 from oracle.attention import ref_attention, ref_attention_rows  # noqa: E402
+from oracle.attention_bwd import ref_attention_bwd  # noqa: E402
 from oracle.mxfp8 import dequantize_mxfp8_ref, quantize_mxfp8_ref  # noqa: E402
 from helpers import BF16_MAX_ABS, BF16_MEAN_ABS, LSE_ABS, MXFP8_MAX_ABS, run_gpu  # noqa: E402
 
@@ -57,7 +61,55 @@ def line(name, rows, e, le, max_tol, mean_tol):
                          and le.max() <= LSE_ABS)}
 
 
+def bwd_lines():
+    import math
+    from test_gpu_bwd import BWD_REL_MAX, BWD_REL_MEAN
+    lines = []
+    cases = [("bwd tiny-shape (L256 H2 d64)", [256], 2, 64),
+             ("bwd ragged packed (7 docs, H2 d64)", [1, 130, 300, 129, 64, 256, 44], 2, 64),
+             ("bwd ragged packed (7 docs, H2 d128)", [1, 130, 300, 129, 64, 256, 44], 2, 128),
+             ("bwd one document L2048 H2 d128", [2048], 2, 128)]
+    dev = torch.device("cuda:0")
+    for name, lengths, H, d in cases:
+        for causal in (True, False):
+            g = torch.Generator().manual_seed(21)
+            T = sum(lengths)
+            q, k, v, do = (torch.randn((T, H, d), generator=g).to(torch.bfloat16)
+                           for _ in range(4))
+            scale = 1.0 / math.sqrt(d)
+            cu = workloads.cu_from_lengths(lengths)
+            qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+            cud = cu.to(dev)
+            out = torch.empty_like(qd)
+            lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+            A.attn_fwd(qd, kd, vd, cud, out, lse, causal, scale, max_seqlen=max(lengths))
+            grads = [torch.empty_like(qd) for _ in range(3)]
+            A.attn_bwd(qd, kd, vd, out, dod, lse, cud, *grads, causal, scale,
+                       max_seqlen=max(lengths))
+            torch.cuda.synchronize()
+            ref = ref_attention_bwd(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                    do.double().numpy(), cu.numpy(), causal, scale)
+            rec = {"config": f"{name}, {'causal' if causal else 'non-causal'}",
+                   "tol_rel": {"max": BWD_REL_MAX, "mean": BWD_REL_MEAN}}
+            ok = True
+            for gname, got, rf in zip(("dq", "dk", "dv"), grads, ref):
+                e = np.abs(got.cpu().double().numpy() - rf)
+                m = float(np.abs(rf).max())
+                rec[gname] = {"max_abs": float(e.max()), "mean_abs": float(e.mean()),
+                              "max_ref": m, "max_rel": float(e.max()) / m,
+                              "mean_rel": float(e.mean()) / m}
+                ok &= e.max() <= BWD_REL_MAX * m and e.mean() <= BWD_REL_MEAN * m
+            rec["pass"] = bool(ok)
+            lines.append(rec)
+    return lines
+
+
 def main():
+    if "--bwd-only" in sys.argv:
+        lines = bwd_lines()
+        for l_ in lines:
+            print(json.dumps(l_))
+        return 0 if all(l_["pass"] for l_ in lines) else 1
     out_lines = []
     inp = workloads.make_inputs("tiny")
     for causal in (False, True):
@@ -87,6 +139,7 @@ def main():
         le = np.abs(lse[heads, toks].double().numpy() - rl)
         out_lines.append(line(name, len(toks), e, le, MXFP8_MAX_ABS if fp8 else BF16_MAX_ABS,
                               None if fp8 else BF16_MEAN_ABS))
+    out_lines += bwd_lines()
     for l_ in out_lines:
         print(json.dumps(l_))
     return 0 if all(l_["pass"] for l_ in out_lines) else 1
