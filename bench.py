@@ -18,7 +18,8 @@ sample of the same workload and prints the same metric (rank 0 only).
 ``--pass bwd`` times the backward instead (bf16 workloads): one step = one
 ``attn_bwd`` call (schedule, D pre-pass, backward kernel, dQ conversion)
 with the forward's out and lse resident; FLOPs = 2.5 x the forward's (five
-products against two); the fp64 gradient oracle is the CPU baseline.
+products against two); the fp64 gradient oracle is the CPU baseline, and
+``--impl reference --pass bwd`` times that oracle the same way.
 """
 from __future__ import annotations
 
@@ -575,16 +576,27 @@ def bench_reference(args):
         return None
     w = workloads.get(args.workload)
     inp = workloads.make_inputs(w)
+    T, H, d = inp["q"].shape
+    bwd = getattr(args, "which", "fwd") == "bwd"
+    if bwd:
+        # the same seeded upstream gradient as the GPU arm
+        dout = torch.randn((T, H, d), generator=torch.Generator().manual_seed(1000 + w.seed))
+        dout = dout.to(torch.bfloat16)
+
+        def sample(budget_s):
+            return cpu_baseline_bwd(inp, dout, budget_s=budget_s)
+    else:
+        def sample(budget_s):
+            return cpu_baseline(w, inp, budget_s=budget_s)
     budget = max(2.0, args.cpu_budget / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_baseline(w, inp, budget_s=budget)
-    vals = [cpu_baseline(w, inp, budget_s=budget) for _ in range(args.steps)]
+        sample(budget)
+    vals = [sample(budget) for _ in range(args.steps)]
     v = round(statistics.median(x["value"] for x in vals), 6)
-    T, H, d = inp["q"].shape
-    flops = workloads.flops(inp["lengths"], H, d, True)
+    flops = (2.5 if bwd else 1.0) * workloads.flops(inp["lengths"], H, d, True)
     return {
         "impl": "reference",
-        "metric": METRIC,
+        "metric": METRIC_BWD if bwd else METRIC,
         "value": v,
         "unit": "TFLOP/s",
         "n_gpus": world,

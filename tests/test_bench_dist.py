@@ -62,3 +62,33 @@ def test_reference_arm_is_rank0_only(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
     args = argparse.Namespace(workload="tiny", steps=1, warmup=3, cpu_budget=1.0)
     assert bench.bench_reference(args) is None
+
+
+@pytest.mark.parametrize("which", ["fwd", "bwd"])
+def test_reference_arm_runs_the_oracle(which, monkeypatch):
+    """Rank 0 of the reference arm times the fp64 oracle (forward, or the
+    gradients with --pass bwd) on the host cores and reports the arm's
+    metric; no GPU is touched."""
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    args = argparse.Namespace(workload="tiny", steps=1, warmup=3, cpu_budget=1.0, which=which)
+    line = bench.bench_reference(args)
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["metric"] == (bench.METRIC_BWD if which == "bwd" else bench.METRIC)
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    factor = 2.5 if which == "bwd" else 1.0
+    assert line["config"]["flops_per_step"] == pytest.approx(
+        factor * 4.0 * 256 * 256 * 64 / 2.0 * 2)
+
+
+def test_forward_source_hash_ignores_the_backward():
+    """The forward's traffic record stays valid when only backward sources
+    change: its hash skips attn_bwd* files and attn_api.cu past the
+    backward marker, and the backward's hash does not."""
+    import bench
+    api = os.path.join(ROOT, "exact_tiled_attention_39_b200", "csrc", "attn_api.cu")
+    data = open(api, "rb").read()
+    assert data.count(bench.BWD_SECTION_MARK) == 1
+    assert bench.kernel_sources_sha256("fwd") != bench.kernel_sources_sha256("bwd")
