@@ -72,9 +72,10 @@ def _compare(lengths, H, d, causal, seed, dense=False):
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [True, False])
 def test_bwd_packed_ragged(d, causal):
-    """Ragged packed documents: a one-token document, tails of 1, 2, 44 and
-    64 rows past a tile edge, an exact tile, several query and key tiles."""
-    _compare([1, 130, 300, 129, 64, 256, 44], 2, d, causal, seed=11)
+    """Ragged packed documents: a one-token document, an empty one, tails of
+    1, 2, 44 and 64 rows past a tile edge, an exact tile, several query and
+    key tiles."""
+    _compare([1, 130, 0, 300, 129, 64, 256, 44], 2, d, causal, seed=11)
 
 
 def test_bwd_dense_batch():
