@@ -53,28 +53,39 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-# attn_api.cu holds the backward's host code after this line; the forward's
-# sources end before it.
+# attn_api.cu holds, after the forward's host code, one section per later
+# part, each opening with one of these marker lines.
 BWD_SECTION_MARK = b"\n// " + b"=" * 75 + b"\n// Backward (bf16)"
+INCOHERENT_SECTION_MARK = b"\n// " + b"=" * 75 + b"\n// Incoherent processing"
+
+# The CUDA sources each measured kernel is built and launched from, and the
+# marker where that part's share of attn_api.cu ends.
+FWD_SOURCES = ["attn_api.cu", "attn_fwd_pair_sm100.cuh", "attn_fwd_sm100.cuh", "common.cuh",
+               "ptx.cuh", "quant_mxfp8.cuh", "schedule.cuh", "tmem_ops.cuh"]
+PART_SOURCES = {
+    "fwd": (FWD_SOURCES, BWD_SECTION_MARK),
+    "bwd": (FWD_SOURCES + ["attn_bwd_sm100.cuh"], INCOHERENT_SECTION_MARK),
+}
 
 
 def kernel_sources_sha256(part: str = "fwd") -> str:
-    """Hash of the CUDA sources (names and bytes) a kernel is built and
-    launched from.  "fwd": every csrc file except the backward's, and
-    attn_api.cu up to its backward section; "bwd": every csrc file."""
+    """Hash of the CUDA sources (names and bytes, sorted by name) a measured
+    kernel is built and launched from: "fwd" the forward kernels, "bwd" the
+    backward (the forward's files, the backward kernel's, and attn_api.cu up
+    to the next part's section)."""
     import hashlib
     d = os.path.join(ROOT, "exact_tiled_attention_39_b200", "csrc")
+    files, end_mark = PART_SOURCES[part]
     h = hashlib.sha256()
-    for n in sorted(os.listdir(d)):
-        if n.endswith((".cu", ".cuh")) and (part == "bwd" or not n.startswith("attn_bwd")):
-            h.update(n.encode())
-            with open(os.path.join(d, n), "rb") as f:
-                data = f.read()
-            if n == "attn_api.cu" and part == "fwd":
-                cut = data.find(BWD_SECTION_MARK)
-                if cut >= 0:
-                    data = data[:cut]
-            h.update(data)
+    for n in sorted(files):
+        h.update(n.encode())
+        with open(os.path.join(d, n), "rb") as f:
+            data = f.read()
+        if n == "attn_api.cu":
+            cut = data.find(end_mark)
+            if cut >= 0:
+                data = data[:cut]
+        h.update(data)
     return h.hexdigest()
 
 

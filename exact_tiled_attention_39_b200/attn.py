@@ -15,7 +15,8 @@ import torch
 __all__ = ["ATTN_BF16", "ATTN_MXFP8", "AttnError", "lib", "workspace_size", "attn_fwd",
            "attn_fwd_noalloc", "attn_quantize_mxfp8", "attn_get_device_error", "status_string",
            "make_workspace", "attn_timing_enable", "attn_timing_read", "bwd_workspace_size",
-           "make_bwd_workspace", "attn_bwd", "LIB_PATH", "EXPORTED_SYMBOLS"]
+           "make_bwd_workspace", "attn_bwd", "attn_quantize_mxfp8_rotated", "LIB_PATH",
+           "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 
@@ -30,7 +31,7 @@ STATUS = {
 EXPORTED_SYMBOLS = ("attn_workspace_size", "attn_fwd", "attn_quantize_mxfp8",
                     "attn_get_device_error", "attn_status_string", "attn_abi_version",
                     "attn_fwd_noalloc", "attn_timing_enable", "attn_timing_read",
-                    "attn_bwd_workspace_size", "attn_bwd")
+                    "attn_bwd_workspace_size", "attn_bwd", "attn_quantize_mxfp8_rotated")
 
 
 class AttnError(RuntimeError):
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
                                ctypes.c_float, ctypes.c_int, vp, ctypes.POINTER(_Shape), vp, sz]
         L.attn_bwd.restype = ctypes.c_int
+        L.attn_quantize_mxfp8_rotated.argtypes = [vp, vp, vp, vp, i64, i32, vp]
+        L.attn_quantize_mxfp8_rotated.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -223,6 +226,19 @@ def attn_quantize_mxfp8(x, codes, scales, stream=None):
                                    _stream_handle(stream, x.device))
     if rc != 0:
         raise AttnError(rc, "attn_quantize_mxfp8")
+
+
+def attn_quantize_mxfp8_rotated(x, signs, codes, scales, stream=None):
+    """Incoherent processing then MXFP8 quantisation of a bf16 [rows, cols]
+    CUDA tensor (cols 64 or 128; any leading shape): signs fp32 [cols] (+-1)
+    on the device; codes uint8 [rows, cols], scales uint8 [rows, cols / 32]
+    (``attn_quantize_mxfp8_rotated``)."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    rc = lib().attn_quantize_mxfp8_rotated(_ptr(x), _ptr(signs), _ptr(codes), _ptr(scales), rows,
+                                           cols, _stream_handle(stream, x.device))
+    if rc != 0:
+        raise AttnError(rc, "attn_quantize_mxfp8_rotated")
 
 
 def attn_timing_enable(enable: bool) -> None:

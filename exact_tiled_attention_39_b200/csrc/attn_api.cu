@@ -597,3 +597,31 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Incoherent processing: attn_quantize_mxfp8_rotated.  The forward's and the
+// backward's sources end above this line.
+// ===========================================================================
+#include "incoherent.cuh"
+
+extern "C" attn_status_t attn_quantize_mxfp8_rotated(const void* x, const float* signs,
+                                                     uint8_t* codes, uint8_t* scales,
+                                                     int64_t rows, int32_t cols, void* stream) {
+  if (rows < 0 || (cols != 64 && cols != 128)) return rows < 0 ? ATTN_ERR_INVALID_ARG
+                                                               : ATTN_ERR_UNSUPPORTED;
+  if (rows == 0) return ATTN_OK;
+  if (x == nullptr || signs == nullptr || codes == nullptr || scales == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u) != 0)
+    return ATTN_ERR_ALIGNMENT;
+  const long long grid = (rows + 127) / 128;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  if (cols == 128)
+    quantize_mxfp8_rotated_kernel<128><<<static_cast<unsigned>(grid), 128, 0, strm>>>(
+        static_cast<const uint4*>(x), signs, reinterpret_cast<uint4*>(codes), scales, rows);
+  else
+    quantize_mxfp8_rotated_kernel<64><<<static_cast<unsigned>(grid), 128, 0, strm>>>(
+        static_cast<const uint4*>(x), signs, reinterpret_cast<uint4*>(codes), scales, rows);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}

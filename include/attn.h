@@ -149,6 +149,22 @@ attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v,
 attn_status_t attn_quantize_mxfp8(const void* x, uint8_t* codes, uint8_t* scales, int64_t rows,
                                   int32_t cols, void* stream);
 
+/* The MXFP8 pre-pass with incoherent processing ("FlashAttention, pelatihan
+ * multi-GPU, dan kuantisasi bobot", section 1: Q and K multiplied by a random
+ * orthogonal matrix before quantisation, to spread outlier channels).  Each
+ * row r of x (bf16 [rows, cols], cols 64 or 128) becomes y = (x_r * s) H
+ * with s = signs (device fp32 [cols], each +1 or -1) and H the unnormalised
+ * Sylvester Hadamard matrix of order cols (H H^T = cols I), computed in fp32
+ * by the fast Walsh-Hadamard butterfly (spans 1, 2, 4, ..., cols / 2; each
+ * pair (a, b) -> (a + b, a - b), round to nearest); y is then quantised as by
+ * attn_quantize_mxfp8.  Rotating both Q and K multiplies every score by
+ * cols, so a caller divides its softmax scale by cols.  codes: uint8
+ * [rows, cols] E4M3, 16-byte aligned; scales: uint8 [rows, cols / 32] E8M0,
+ * 4-byte aligned.  ATTN_ERR_UNSUPPORTED for other cols.  Asynchronous. */
+attn_status_t attn_quantize_mxfp8_rotated(const void* x, const float* signs, uint8_t* codes,
+                                          uint8_t* scales, int64_t rows, int32_t cols,
+                                          void* stream);
+
 /* Synchronises `stream`, then reads the workspace's error word into
  * *device_status and clears it.  The word holds the outcome of the most
  * recent attn_fwd on this workspace (each call resets it when it starts):

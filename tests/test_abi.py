@@ -138,3 +138,13 @@ def test_bwd_host_checks_return_before_launch(L):
     assert _bwd(L, ok, ws=0) == 4
     assert _bwd(L, ok, ws_bytes=64) == 4
     assert _bwd(L, A.Shape(0, 0, 2, 64, 0)) == 0                # T == 0: no-op
+
+
+def test_rotated_quantiser_host_checks(L):
+    vp = ctypes.c_void_p
+    assert L.attn_quantize_mxfp8_rotated(None, None, None, None, 0, 128, None) == 0   # empty
+    assert L.attn_quantize_mxfp8_rotated(None, None, None, None, 4, 96, None) == 2    # cols
+    assert L.attn_quantize_mxfp8_rotated(None, None, None, None, -1, 128, None) == 1
+    assert L.attn_quantize_mxfp8_rotated(vp(16), None, vp(16), vp(16), 4, 128, None) == 1
+    assert L.attn_quantize_mxfp8_rotated(vp(16), vp(16), vp(24), vp(16), 4, 64, None) == 3
+    assert L.attn_quantize_mxfp8_rotated(vp(16), vp(16), vp(16), vp(18), 4, 64, None) == 3
