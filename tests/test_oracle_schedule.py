@@ -59,3 +59,29 @@ def test_unit_cost_edges():
     assert unit_cost(129, 0, True, 2) == 3
     assert unit_cost(256, 0, False, 2) == 4
     assert unit_cost(257, 1, True, 2) == 3
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_reads_the_list_as_key_tiles(causal):
+    """The backward takes each entry (doc_start, doc_len, t, cost) of the
+    one-tile list as key tile kb = n_tiles - 1 - t of that document.  Counted
+    by brute force over (query tile, key tile) pairs of the mask: the key
+    tiles so obtained are each document's key tiles exactly once, and an
+    entry's cost is the number of query tiles that see its key tile, so the
+    list stays heaviest first for the backward's units."""
+    lengths = [1, 300, 0, 128, 129, 1000, 64]
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    lst = schedule_ref(cu, causal, 1)
+    seen = set()
+    for a, L, t, cost in lst:
+        n = -(-int(L) // 128)
+        kb = n - 1 - int(t)
+        assert 0 <= kb < n
+        assert (int(a), kb) not in seen
+        seen.add((int(a), kb))
+        # query tiles qb with some query i >= some key j of tile kb (causal),
+        # or any query tile (not causal), inside the document
+        sees = sum(1 for qb in range(n)
+                   if not causal or min(128 * qb + 127, int(L) - 1) >= 128 * kb)
+        assert sees == int(cost)
+    assert len(seen) == sum(-(-L // 128) for L in lengths)
