@@ -23,14 +23,28 @@ and so contribute nothing; a row that sees no key has P = 0 and all its
 gradients are 0.
 
 Layouts as the forward oracle: q, k, v, dout and the results are [T, H, d].
+
+MXFP8 (``ref_attention_bwd_mxfp8``).  FLAMIA (section "FLAMIA Mimarisi ve
+Temel Tasarım İlkeleri") asks for the forward and backward passes to agree
+numerically, for quantised operands reused across orientations, and for
+scales that carry no information from future tokens.  Reading taken: the
+backward differentiates exactly what the MXFP8 forward computed, so it runs
+on the same quantised operands: Q, K, V quantised per (token, head, 32
+head-dim elements) and exactly dequantised, as in the forward oracle; the
+upstream gradient dO quantised the same way; gradients with respect to the
+dequantised operands, passed straight through the quantiser.  Every scale
+covers one token of one head, so none crosses a document or causal
+boundary, and the dequantised values serve every orientation of every
+product unchanged.
 """
 from __future__ import annotations
 
 import numpy as np
 
 from .attention import doc_bounds, ref_probabilities
+from .mxfp8 import dequantize_mxfp8_ref, quantize_mxfp8_ref
 
-__all__ = ["ref_attention_bwd"]
+__all__ = ["ref_attention_bwd", "ref_attention_bwd_mxfp8"]
 
 
 def ref_attention_bwd(q, k, v, dout, cu_seqlens, causal: bool, scale: float):
@@ -57,3 +71,13 @@ def ref_attention_bwd(q, k, v, dout, cu_seqlens, causal: bool, scale: float):
             dq[a:b, h] = scale * (ds @ kh)
             dk[a:b, h] = scale * (ds.T @ qh)
     return dq, dk, dv
+
+
+def ref_attention_bwd_mxfp8(q, k, v, dout, cu_seqlens, causal: bool, scale: float):
+    """(dq, dk, dv) of the MXFP8 path, fp64 [T, H, d]: the gradients above
+    on the exactly dequantised MXFP8 operands (q, k, v and dout quantised
+    per token, head and 32 head-dim elements)."""
+    def deq(x):
+        return dequantize_mxfp8_ref(*quantize_mxfp8_ref(np.asarray(x, dtype=np.float64)))
+
+    return ref_attention_bwd(deq(q), deq(k), deq(v), deq(dout), cu_seqlens, causal, scale)
