@@ -100,3 +100,36 @@ def test_scales_are_per_token():
     np.testing.assert_array_equal(c0[keep], c1[keep])
     np.testing.assert_array_equal(s0[keep], s1[keep])
     assert not np.array_equal(s0[17], s1[17])
+
+
+def test_encode_matches_brute_force_search():
+    """Every finite magnitude's code by exhaustive search over the 256-code
+    table, written independently of the encoder: the nearest finite value,
+    an exact tie going to the code whose last bit is 0, magnitudes past 448
+    to 448; the sign bit set for negative inputs.  Random magnitudes over
+    the whole range, every midpoint between neighbours (the ties), the
+    neighbours themselves and values past saturation."""
+    from oracle.mxfp8 import e4m3_decode_table, e4m3_encode
+
+    table = e4m3_decode_table()
+    finite = [(c, table[c]) for c in range(128) if np.isfinite(table[c])]
+
+    def brute(x):
+        a = abs(x)
+        if a >= 448.0:
+            code = max(c for c, v in finite if v == 448.0)
+        else:
+            best = min(abs(v - a) for _, v in finite)
+            cands = [c for c, v in finite if abs(v - a) == best]
+            code = min(cands, key=lambda c: (c & 1, c))
+        return code | (0x80 if np.signbit(x) else 0)
+
+    vals = sorted(v for _, v in finite)
+    mids = [(a + b) / 2 for a, b in zip(vals[:-1], vals[1:])]
+    rng = np.random.default_rng(17)
+    rand = np.exp(rng.uniform(np.log(1e-4), np.log(600.0), 400))
+    xs = np.concatenate([rand, mids, vals, [448.0, 460.0, 1e4, 0.0]])
+    xs = np.concatenate([xs, -xs])
+    got = e4m3_encode(xs)
+    want = np.array([brute(float(x)) for x in xs], dtype=np.uint8)
+    np.testing.assert_array_equal(got, want)
