@@ -250,3 +250,29 @@ def test_row_chunking_does_not_change_result():
     o2, l2 = ref_attention(q, k, v, cu, True, 0.3, row_chunk=4096)
     np.testing.assert_allclose(o1, o2, atol=1e-15)
     np.testing.assert_allclose(l1, l2, atol=1e-15)
+
+
+def test_online_replay_any_partition_and_order():
+    """The running statistics reach the direct softmax-weighted sum for any
+    partition of the keys into blocks and any block order (the recurrence's
+    exactness claim), including blocks whose maximum is below the running
+    one, a block holding the row maximum last, and scores far apart
+    (exp(-100) weights); the final l is the direct sum of exp(s - max)."""
+    rng = np.random.default_rng(23)
+    for trial in range(40):
+        n = int(rng.integers(1, 40))
+        s = rng.normal(0.0, 3.0, n)
+        if trial % 4 == 0:
+            s[int(rng.integers(0, n))] += 100.0        # one dominant key
+        v = rng.normal(size=(n, 5))
+        perm = rng.permutation(n)
+        cuts = np.sort(rng.choice(np.arange(1, n), size=min(n - 1, int(rng.integers(0, 6))),
+                                  replace=False)) if n > 1 else []
+        blocks = [list(b) for b in np.split(perm, cuts)]
+        got, trace = online_replay(s, v, blocks)
+        w = np.exp(s - s.max())
+        want = (w[:, None] * v).sum(0) / w.sum()
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-13)
+        m_final, l_final, _ = trace[-1]
+        assert m_final == s.max()
+        np.testing.assert_allclose(l_final, w.sum(), rtol=1e-13)
