@@ -134,40 +134,47 @@ def attn_fwd(q, k, v, cu_seqlens, out, lse, causal: bool, scale: float, dtype: i
     cu_seqlens, ``max_seqlen`` must bound every document length (a longer
     one is reported by the device as ATTN_ERR_BAD_SEQLENS).  Returns the
     workspace used (allocated if not given)."""
-    T, H, d = q.shape
-    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.shape != q.shape:
-            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
-    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (H, T):
-        raise ValueError("lse must be a contiguous fp32 tensor of shape [H, T]")
-    if cu_seqlens is not None:
-        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
-            raise ValueError("cu_seqlens must be an int32 CUDA tensor")
-        ns = cu_seqlens.numel() - 1
-        if max_seqlen is None:
-            raise ValueError("max_seqlen is required with cu_seqlens (no host sync is done)")
-    else:
-        ns = num_seqs if num_seqs is not None else 1
-        if max_seqlen is None:
-            max_seqlen = T // max(ns, 1)
-    shape = Shape(T, ns, H, d, int(max_seqlen))
-    if workspace is None:
-        workspace = make_workspace(shape, dtype, q.device)
-    s = shape.c()
-    rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(out), _ptr(lse),
-                        int(bool(causal)), float(scale), int(dtype),
-                        _stream_handle(stream, q.device), ctypes.byref(s), _ptr(workspace),
-                        workspace.numel())
+    shape = _check_fwd_args(q, k, v, out, lse, cu_seqlens, max_seqlen, num_seqs)
+    with torch.cuda.device(q.device):
+        if workspace is None:
+            workspace = make_workspace(shape, dtype, q.device)
+        elif not workspace.is_cuda or workspace.device != q.device:
+            raise ValueError("workspace must be on the same CUDA device as q")
+        s = shape.c()
+        rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(out), _ptr(lse),
+                            int(bool(causal)), float(scale), int(dtype),
+                            _stream_handle(stream, q.device), ctypes.byref(s), _ptr(workspace),
+                            workspace.numel())
     if rc != 0:
         raise AttnError(rc, "attn_fwd")
     return workspace
 
 
+def _check_fwd_args(q, k, v, out, lse, cu_seqlens, max_seqlen, num_seqs) -> Shape:
+    """Checks shared by the forward entry points; returns the problem shape.
+    Every tensor must be on q's CUDA device: the library launches on the
+    device that is current during the call, which the callers set to q's."""
+    if q.dim() != 3:
+        raise ValueError("q must have shape [T, H, d]")
+    T, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        if (t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous()
+                or t.shape != q.shape or t.device != q.device):
+            raise ValueError(f"{name} must be a contiguous bf16 tensor of shape "
+                             f"{tuple(q.shape)} on {q.device}")
+    if (lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous()
+            or tuple(lse.shape) != (H, T) or lse.device != q.device):
+        raise ValueError(f"lse must be a contiguous fp32 tensor of shape [H, T] on {q.device}")
+    return _doc_shape(q, cu_seqlens, max_seqlen, num_seqs)
+
+
 def _doc_shape(q, cu_seqlens, max_seqlen, num_seqs) -> Shape:
     T, H, d = q.shape
     if cu_seqlens is not None:
-        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
-            raise ValueError("cu_seqlens must be an int32 CUDA tensor")
+        if (cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda
+                or not cu_seqlens.is_contiguous() or cu_seqlens.dim() != 1
+                or cu_seqlens.device != q.device):
+            raise ValueError(f"cu_seqlens must be a contiguous 1-D int32 tensor on {q.device}")
         ns = cu_seqlens.numel() - 1
         if max_seqlen is None:
             raise ValueError("max_seqlen is required with cu_seqlens (no host sync is done)")
@@ -192,7 +199,7 @@ def make_bwd_workspace(shape: Shape, device=None) -> torch.Tensor:
 
 def attn_bwd(q, k, v, out, dout, lse, cu_seqlens, dq, dk, dv, causal: bool, scale: float,
              stream=None, workspace=None, max_seqlen: int | None = None,
-             num_seqs: int | None = None):
+             num_seqs: int | None = None, dtype: int = ATTN_BF16):
     """Gradients of the forward through the C ABI (``attn_bwd``): q, k, v,
     out (the forward's output), dout: bf16 [T, H, d]; lse: fp32 [H, T] from
     the forward; dq, dk, dv: bf16 [T, H, d], written.  Same document rules
@@ -200,18 +207,24 @@ def attn_bwd(q, k, v, out, dout, lse, cu_seqlens, dq, dk, dv, causal: bool, scal
     T, H, d = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("dq", dq),
                     ("dk", dk), ("dv", dv)):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.shape != q.shape:
-            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
-    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (H, T):
-        raise ValueError("lse must be a contiguous fp32 tensor of shape [H, T]")
+        if (t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous()
+                or t.shape != q.shape or t.device != q.device):
+            raise ValueError(f"{name} must be a contiguous bf16 tensor of shape "
+                             f"{tuple(q.shape)} on {q.device}")
+    if (lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous()
+            or tuple(lse.shape) != (H, T) or lse.device != q.device):
+        raise ValueError(f"lse must be a contiguous fp32 tensor of shape [H, T] on {q.device}")
     shape = _doc_shape(q, cu_seqlens, max_seqlen, num_seqs)
-    if workspace is None:
-        workspace = make_bwd_workspace(shape, q.device)
-    s = shape.c()
-    rc = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
-                        _ptr(cu_seqlens), _ptr(dq), _ptr(dk), _ptr(dv), int(bool(causal)),
-                        float(scale), ATTN_BF16, _stream_handle(stream, q.device),
-                        ctypes.byref(s), _ptr(workspace), workspace.numel())
+    with torch.cuda.device(q.device):
+        if workspace is None:
+            workspace = make_bwd_workspace(shape, q.device)
+        elif not workspace.is_cuda or workspace.device != q.device:
+            raise ValueError("workspace must be on the same CUDA device as q")
+        s = shape.c()
+        rc = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                            _ptr(cu_seqlens), _ptr(dq), _ptr(dk), _ptr(dv), int(bool(causal)),
+                            float(scale), int(dtype), _stream_handle(stream, q.device),
+                            ctypes.byref(s), _ptr(workspace), workspace.numel())
     if rc != 0:
         raise AttnError(rc, "attn_bwd")
     return workspace
@@ -279,17 +292,11 @@ def attn_fwd_noalloc(q, k, v, cu_seqlens, out, lse, causal: bool, scale: float, 
     fn.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_float, vp,
                    ctypes.POINTER(_Shape)]
     fn.restype = ctypes.c_int
-    T, H, d = q.shape
-    if cu_seqlens is not None:
-        ns = cu_seqlens.numel() - 1
-        if max_seqlen is None:
-            raise ValueError("max_seqlen is required with cu_seqlens (no host sync is done)")
-    else:
-        ns = num_seqs if num_seqs is not None else 1
-        if max_seqlen is None:
-            max_seqlen = T // max(ns, 1)
-    s = Shape(T, ns, H, d, int(max_seqlen)).c()
-    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(out), _ptr(lse),
-            int(bool(causal)), float(scale), _stream_handle(stream, q.device), ctypes.byref(s))
+    s = _check_fwd_args(q, k, v, out, lse, cu_seqlens, max_seqlen, num_seqs).c()
+    # The library looks up its scratch on the current device: make that q's.
+    with torch.cuda.device(q.device):
+        rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(out), _ptr(lse),
+                int(bool(causal)), float(scale), _stream_handle(stream, q.device),
+                ctypes.byref(s))
     if rc != 0:
         raise AttnError(rc, "attn_fwd_noalloc")

@@ -8,6 +8,7 @@ at load time.
 """
 from __future__ import annotations
 
+import hashlib
 import os
 import shutil
 import subprocess
@@ -39,16 +40,44 @@ def sources() -> list[str]:
                   if f.endswith((".cu", ".cuh")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def _deps() -> list[str]:
+    return sources() + [os.path.join(ROOT, "include", "attn.h"), __file__]
+
+
+def source_hash(defines: dict[str, str] | None = None) -> str:
+    """SHA-256 over the names and bytes of every file the library is built
+    from, the compiler flags and any extra defines."""
+    h = hashlib.sha256()
+    for path in _deps():
+        h.update(os.path.relpath(path, ROOT).encode())
+        with open(path, "rb") as f:
+            h.update(f.read())
+    h.update(repr(NVCC_FLAGS).encode())
+    h.update(repr(sorted((defines or {}).items())).encode())
+    return h.hexdigest()
+
+
+def _stamp(lib_path: str) -> str:
+    return lib_path + ".src-sha256"
+
+
+def _current(lib_path: str, digest: str) -> bool:
+    """True when lib_path exists and was built from sources with this hash
+    (recorded in a stamp file beside it).  File times are not trusted: a
+    copied tree can carry a binary newer than its sources."""
+    if not os.path.exists(lib_path) or not os.path.exists(_stamp(lib_path)):
         return False
-    t = os.path.getmtime(LIB)
-    deps = sources() + [os.path.join(ROOT, "include", "attn.h"), __file__]
-    return all(os.path.getmtime(s) <= t for s in deps)
+    with open(_stamp(lib_path)) as f:
+        return f.read().strip() == digest
+
+
+def up_to_date() -> bool:
+    return _current(LIB, source_hash())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+    digest = source_hash()
+    if not force and _current(LIB, digest):
         return LIB
     cmd = [_nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"),
            os.path.join(CSRC, "attn_api.cu"), "-o", LIB + ".tmp"]
@@ -58,6 +87,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if res.returncode != 0:
         raise RuntimeError("nvcc failed building libattn.so")
     os.replace(LIB + ".tmp", LIB)
+    with open(_stamp(LIB), "w") as f:
+        f.write(digest + "\n")
     with open(os.path.join(PKG, "build_ptxas.log"), "w") as f:
         f.write(res.stderr)
     return LIB
@@ -65,11 +96,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 def build_variant(name: str, defines: dict[str, str]) -> str:
     """Build ``libattn_<name>.so`` in-tree with extra preprocessor defines
-    (test builds: the failure-detection test uses one); rebuilt when a source
-    is newer."""
+    (test builds: the failure-detection test uses one); rebuilt when the
+    source hash differs from the one recorded beside it."""
     out = os.path.join(PKG, f"libattn_{name}.so")
-    deps = sources() + [os.path.join(ROOT, "include", "attn.h"), __file__]
-    if os.path.exists(out) and all(os.path.getmtime(s) <= os.path.getmtime(out) for s in deps):
+    digest = source_hash(defines)
+    if _current(out, digest):
         return out
     cmd = [_nvcc(), *[f for f in NVCC_FLAGS if f not in ("-Xptxas", "-v")],
            *[f"-D{k}={v}" for k, v in defines.items()], "-I", os.path.join(ROOT, "include"),
@@ -79,6 +110,8 @@ def build_variant(name: str, defines: dict[str, str]) -> str:
         sys.stderr.write(res.stdout + res.stderr)
         raise RuntimeError(f"nvcc failed building libattn_{name}.so")
     os.replace(out + ".tmp", out)
+    with open(_stamp(out), "w") as f:
+        f.write(digest + "\n")
     return out
 
 

@@ -104,7 +104,8 @@ constexpr int kPolyPairPeriod = ATTN_POLY_PAIR_PERIOD;
 
 
 // 2^f on [0, 1): 1 + f (c1 + f (c2 + f c3)), a minimax fit of the relative
-// error (max 8.6e-5) made by csrc/fit_exp2_poly.py; p(0) = 1 exactly.
+// error (max 8.6e-5), found by linear programming over a dense grid of
+// [0, 1) with the constant term fixed at 1, so p(0) = 1 exactly.
 constexpr float kExp2C1 = 6.951168180e-01f;
 constexpr float kExp2C2 = 2.276448607e-01f;
 constexpr float kExp2C3 = 7.706713676e-02f;

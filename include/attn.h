@@ -66,7 +66,10 @@ extern "C" {
 typedef enum {
   ATTN_BF16 = 0,  /* bf16 operands, bf16 tensor-core products, fp32 softmax   */
   ATTN_MXFP8 = 1  /* bf16 inputs quantised in-call to E4M3 + E8M0 (per token,
-                     head and 32 head-dim elements), block-scaled products    */
+                     head and 32 head-dim elements).  d = 128: Q K^T is a
+                     block-scaled E4M3 product; P V runs in bf16 on the exact
+                     dequantisation of V.  d = 64: every product runs in bf16
+                     on the exactly dequantised Q, K and V (same values)     */
 } attn_dtype_t;
 
 typedef enum {

@@ -61,6 +61,42 @@ def test_no_alloc_matches_workspace_entry_point_twice():
         assert torch.isfinite(out.float()).all()
 
 
+def _edge_pack(n_short, long_len):
+    """n_short one-token documents then one of long_len tokens (1 head, d 64)."""
+    return [1] * n_short + [long_len]
+
+
+def test_no_alloc_size_limit_edges():
+    """The fixed scratch holds the work lists of problems with
+    total_tokens / 128 + num_seqs <= 32751 (integer division).  A problem
+    exactly at that edge runs and matches attn_fwd; one past it is rejected
+    on the host with ATTN_ERR_WORKSPACE before anything is launched."""
+    dev = torch.device("cuda:0")
+    # at the edge: 32494 + 1 documents, 32768 tokens -> 256 + 32495 = 32751
+    lengths = _edge_pack(32494, 274)
+    assert sum(lengths) // 128 + len(lengths) == 32751
+    q, k, v, cu = _pack(lengths, 1, 64, seed=13)
+    T = q.shape[0]
+    ref_out = torch.empty_like(q)
+    ref_lse = torch.empty((1, T), dtype=torch.float32, device=dev)
+    ws = A.attn_fwd(q, k, v, cu, ref_out, ref_lse, True, 0.125, max_seqlen=274)
+    assert A.attn_get_device_error(ws) == 0
+    out = torch.full_like(q, float("nan"))
+    lse = torch.full((1, T), float("nan"), dtype=torch.float32, device=dev)
+    A.attn_fwd_noalloc(q, k, v, cu, out, lse, True, 0.125, max_seqlen=274)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
+    assert torch.equal(lse.view(torch.int32), ref_lse.view(torch.int32))
+    # one past the edge: 32495 + 1 documents, 32768 tokens -> 32752
+    lengths = _edge_pack(32495, 273)
+    assert sum(lengths) // 128 + len(lengths) == 32752
+    q, k, v, cu = _pack(lengths, 1, 64, seed=14)
+    lse = torch.empty((1, q.shape[0]), dtype=torch.float32, device=dev)
+    with pytest.raises(A.AttnError) as ei:
+        A.attn_fwd_noalloc(q, k, v, cu, torch.empty_like(q), lse, True, 0.125, max_seqlen=273)
+    assert ei.value.code == 4
+
+
 def test_no_alloc_rejects_problems_beyond_its_scratch():
     x = torch.empty((8, 1, 64), dtype=torch.bfloat16, device="cuda:0")
     lse = torch.empty((1, 8), dtype=torch.float32, device="cuda:0")
@@ -70,3 +106,25 @@ def test_no_alloc_rejects_problems_beyond_its_scratch():
     with pytest.raises(A.AttnError) as ei:
         A.attn_fwd_noalloc(x, x, x, cu, x, lse, True, 0.125, max_seqlen=8)
     assert ei.value.code == 4
+
+
+@pytest.mark.parametrize("bad", ["lse_shape", "lse_dtype", "out_dtype", "q_noncontig", "cu_dtype"])
+def test_no_alloc_binding_rejects_bad_tensors(bad):
+    """The binding checks every tensor before the call: a wrong shape, type
+    or layout would otherwise let the kernel write out of bounds."""
+    dev = torch.device("cuda:0")
+    q, k, v, cu = _pack([100, 28], 2, 64, seed=15)
+    out = torch.empty_like(q)
+    lse = torch.empty((2, 128), dtype=torch.float32, device=dev)
+    if bad == "lse_shape":
+        lse = torch.empty((2, 127), dtype=torch.float32, device=dev)
+    elif bad == "lse_dtype":
+        lse = torch.empty((2, 128), dtype=torch.float16, device=dev)
+    elif bad == "out_dtype":
+        out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    elif bad == "q_noncontig":
+        q = torch.empty((2, 128, 64), dtype=torch.bfloat16, device=dev).transpose(0, 1)
+    else:
+        cu = cu.to(torch.int64)
+    with pytest.raises(ValueError):
+        A.attn_fwd_noalloc(q, k, v, cu, out, lse, True, 0.125, max_seqlen=100)
