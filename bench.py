@@ -203,15 +203,25 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def bench_ours(args):
-    from exact_tiled_attention_39_b200 import attn as A
+KERNEL_TIMING_LAUNCHES = 50       # per-kernel time: median of at least this many launches
+KERNEL_TIMING_MIN_S = 1.0         # ... and of at least this much device time (clock samples)
+EXTRA_WORKLOADS = ("packed_causal", "long_outlier", "mxfp8_packed")
 
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pg = init_group("nccl", dev)
 
-    w = workloads.get(args.workload)
+def kernel_name_for(dtype_name: str) -> str:
+    """bf16 runs the two-query-tile kernel, MXFP8 (head dim 128) the
+    block-scaled one."""
+    return "attn_fwd_kernel" if dtype_name == "mxfp8" else "attn_fwd_pair_kernel"
+
+
+def measure_workload(A, name, steps, warmup, dev, stream, pg):
+    """Time one workload: `steps` back-to-back attn_fwd calls (device events,
+    barrier + synchronize on both sides, max over ranks), then the attention
+    kernel alone (CUDA events the library records on the launching stream
+    around that kernel; median over at least KERNEL_TIMING_LAUNCHES launches
+    and KERNEL_TIMING_MIN_S of device time).  Returns the figures and the
+    device tensors for the end-to-end leg."""
+    w = workloads.get(name)
     inp = workloads.make_inputs(w)
     T, H, d = inp["q"].shape
     causal = True
@@ -219,55 +229,103 @@ def bench_ours(args):
     lengths = inp["lengths"]
     max_seqlen = max(lengths)
     flops = workloads.flops(lengths, H, d, causal)
-
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     cu = inp["cu_seqlens"].to(dev)
     out = torch.empty_like(q)
     lse = torch.empty((H, T), dtype=torch.float32, device=dev)
     ws = A.make_workspace(A.Shape(T, len(lengths), H, d, max_seqlen), dtype, dev)
-    stream = torch.cuda.current_stream(dev)
 
     def step():
         A.attn_fwd(q, k, v, cu, out, lse, causal, inp["scale"], dtype=dtype, stream=stream,
                    workspace=ws, max_seqlen=max_seqlen)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
-    assert A.attn_get_device_error(ws) == 0, "device error during warm-up"
+    assert A.attn_get_device_error(ws) == 0, f"device error during warm-up ({name})"
 
-    # ---- device-timed region: K steps, barrier + sync on both sides
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for _ in range(args.steps):
-            step()
-        t1.record(stream)
-        torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
     ms_total = max_over_ranks(pg, t0.elapsed_time(t1), dev)
-    ms_step = ms_total / args.steps
+    ms_step = ms_total / steps
     err = A.attn_get_device_error(ws)
-    value = aggregate_tflops(world, flops, ms_step)
 
-    # ---- the attention kernel alone (roofline): CUDA events the library
-    # records on the launching stream around that kernel inside attn_fwd
     A.attn_timing_enable(True)
     per, pre = [], []
-    for _ in range(5):
+    while len(per) < KERNEL_TIMING_LAUNCHES or sum(per) < 1e3 * KERNEL_TIMING_MIN_S:
         step()
         a_ms, p_ms = A.attn_timing_read()
         per.append(a_ms)
         pre.append(p_ms)
+        if len(per) >= 20000:
+            break
     A.attn_timing_enable(False)
     torch.cuda.synchronize(dev)
-    per_ms = statistics.median(per)
-    pre_ms = statistics.median(pre)
+    return {
+        "w": w, "inp": inp, "dtype": dtype, "flops": flops, "ms_total": ms_total,
+        "ms_step": ms_step, "kernel_ms": statistics.median(per),
+        "prepass_ms": statistics.median(pre), "launches_timed": len(per), "err": err,
+        "tensors": (q, k, v, cu, out, lse), "step": step,
+        "launches_per_step": 3 if dtype == A.ATTN_MXFP8 else 2,
+    }
+
+
+def roofline_for(m, peaks, peak_src):
+    """Roofline of the attention kernel: algorithmic FLOPs / its median
+    launch time against the measured dense peak of its dtype (fp8 = 2 x the
+    bf16 figure, the nominal ratio)."""
+    peak_key = "bf16_tflops_sustained" if m["ms_total"] * 1e-3 > 1.0 else "bf16_tflops"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    fp8 = m["w"].dtype == "mxfp8"
+    if fp8:
+        peak *= 2.0
+    achieved = m["flops"] / (m["kernel_ms"] * 1e-3) / 1e12
+    kernel = kernel_name_for(m["w"].dtype)
+    return {
+        "bound": "tensor",
+        "achieved": round(achieved, 2),
+        "peak": peak,
+        "unit": "TFLOP/s",
+        "frac": round(achieved / peak, 4),
+        "peak_source": f"{peak_source_name(peak_key, 1 if fp8 else 0)} ({peak_src})",
+        "timed_unit": (f"attention kernel alone (CUDA events around its launch), median of "
+                       f"{m['launches_timed']} launches"),
+        "kernel_ms": round(m["kernel_ms"], 4),
+        "prepass_ms": round(m["prepass_ms"], 4),
+        "kernel": kernel,
+        "traffic": recorded_traffic(m["w"].name, kernel),
+        "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
+    }
+
+
+def bench_ours(args):
+    from exact_tiled_attention_39_b200 import attn as A
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = init_group("nccl", dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+
+    with ClockSampler(local) as clk:
+        m = measure_workload(A, args.workload, args.steps, args.warmup, dev, stream, pg)
+    w, inp, dtype, flops = m["w"], m["inp"], m["dtype"], m["flops"]
+    q, k, v, cu, out, lse = m["tensors"]
+    step = m["step"]
+    T, H, d = inp["q"].shape
+    lengths = inp["lengths"]
+    value = aggregate_tflops(world, flops, m["ms_step"])
 
     # ---- end to end through the public API: pinned host in, host out
     hq, hk, hv = (inp[n].pin_memory() for n in ("q", "k", "v"))
@@ -299,23 +357,39 @@ def bench_ours(args):
     e2e_ms = max_over_ranks(pg, s0.elapsed_time(s1) / e2e_steps, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcu))
     d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+    roof = roofline_for(m, peaks, peak_src)
+    ms_step, err = m["ms_step"], m["err"]
+    del m, q, k, v, cu, out, lse, step, e2e_step, hq, hk, hv, hout, hlse
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads of the metric (packed, long context, MXFP8):
+    # same protocol, reported beside the headline
+    extra = {}
+    if not args.no_extra_workloads and args.workload == "dense_causal":
+        for name in EXTRA_WORKLOADS:
+            with ClockSampler(local) as xclk:
+                mx = measure_workload(A, name, args.steps, args.warmup, dev, stream, pg)
+            extra[name] = {
+                "workload": f"{name}: {mx['w'].description}",
+                "dtype": mx["w"].dtype,
+                "tokens": mx["inp"]["tokens"], "heads": mx["inp"]["q"].shape[1],
+                "docs": len(mx["inp"]["lengths"]), "flops_per_step": mx["flops"],
+                "ms_per_step": round(mx["ms_step"], 4),
+                "value": round(aggregate_tflops(world, mx["flops"], mx["ms_step"]), 2),
+                "unit": "TFLOP/s",
+                "roofline": roofline_for(mx, peaks, peak_src),
+                "clocks": xclk.summary(),
+                "device_error": mx["err"],
+                "gpu_launches": args.steps * mx["launches_per_step"],
+            }
+            del mx
+            torch.cuda.empty_cache()
 
     if pg:
         pg.barrier()
         pg.destroy_process_group()
     if rank != 0:
         return None
-
-    peaks, peak_src = load_peaks()
-    timed_s = ms_total * 1e-3
-    peak_key = "bf16_tflops_sustained" if timed_s > 1.0 else "bf16_tflops"
-    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
-    if dtype == A.ATTN_MXFP8:
-        peak *= 2.0        # fp8 dense peak = 2 x bf16 (nominal ratio)
-    achieved = flops / (per_ms * 1e-3) / 1e12
-    # bf16 runs the two-query-tile kernel, MXFP8 (head dim 128) the
-    # block-scaled one-tile kernel
-    kernel_name = "attn_fwd_kernel" if dtype == A.ATTN_MXFP8 else "attn_fwd_pair_kernel"
 
     line = {
         "metric": METRIC,
@@ -330,27 +404,8 @@ def bench_ours(args):
         "vs_baseline": None,
         "dtype": "mxfp8" if dtype == A.ATTN_MXFP8 else "bf16",
         "data": "synthetic (seeded N(0,1) bf16, see workloads.py)",
-        "config": {
-            "workload": f"{w.name}: {w.description}",
-            "tokens": T, "heads": H, "head_dim": d, "docs": len(lengths),
-            "causal": causal, "flops_per_step": flops,
-            "l2": f"inputs {3 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2; no flush",
-            "parallelism": f"replicas x{world}",
-        },
-        "roofline": {
-            "bound": "tensor",
-            "achieved": round(achieved, 2),
-            "peak": peak,
-            "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4),
-            "peak_source": f"{peak_source_name(peak_key, dtype)} ({peak_src})",
-            "timed_unit": "attention kernel alone (CUDA events around its launch), median of 5",
-            "kernel_ms": round(per_ms, 4),
-            "prepass_ms": round(pre_ms, 4),
-            "kernel": kernel_name,
-            "traffic": recorded_traffic(w.name, kernel_name),
-            "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
-        },
+        "config": workload_config(w, inp, world),
+        "roofline": roof,
         "e2e": {
             "value": round(aggregate_tflops(world, flops, e2e_ms), 2),
             "unit": "TFLOP/s",
@@ -362,9 +417,25 @@ def bench_ours(args):
         "clocks": clk.summary(),
         "device_error": err,
     }
+    if extra:
+        line["workloads"] = extra
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_budget)
+        cb = cpu_baseline(w, inp, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {key: cb[key] for key in ("value", "unit", "cores", "kind",
+                                                         "sample")}
     return line
+
+
+def workload_config(w, inp, world: int) -> dict:
+    """The `config` object of a workload's line (the same keys in both arms)."""
+    T, H, d = inp["q"].shape
+    return {
+        "workload": f"{w.name}: {w.description}",
+        "tokens": T, "heads": H, "head_dim": d, "docs": len(inp["lengths"]),
+        "causal": True, "flops_per_step": workloads.flops(inp["lengths"], H, d, True),
+        "l2": f"inputs {3 * T * H * d * 2 / 1e6:.0f} MB > 126 MB L2; no flush",
+        "parallelism": f"replicas x{world}",
+    }
 
 
 def peak_source_name(key, dtype):
@@ -403,7 +474,7 @@ def cpu_baseline(w, inp, budget_s=15.0):
     return {"value": round(done_flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
             "kind": "oracle",
             "sample": f"{done} of {len(problems)} (document, head) problems, fp64, "
-                      f"{el:.1f} s"}
+                      f"{el:.1f} s", "seconds": el, "problems": done}
 
 
 def cpu_baseline_bwd(inp, dout, budget_s=15.0):
@@ -431,7 +502,7 @@ def cpu_baseline_bwd(inp, dout, budget_s=15.0):
     return {"value": round(done_flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
             "kind": "oracle",
             "sample": f"{done} of {len(problems)} (document, head) problems, fp64 gradients, "
-                      f"{el:.1f} s"}
+                      f"{el:.1f} s", "seconds": el, "problems": done}
 
 
 def bench_ours_bwd(args):
@@ -546,13 +617,9 @@ def bench_ours_bwd(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16, see workloads.py; dout seeded N(0,1))",
-        "config": {
-            "workload": f"{w.name} backward: {w.description}",
-            "tokens": T, "heads": H, "head_dim": d, "docs": len(lengths),
-            "causal": causal, "flops_per_step": flops,
-            "l2": f"inputs {6 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2; no flush",
-            "parallelism": f"replicas x{world}",
-        },
+        "config": dict(workload_config(w, inp, world),
+                       workload=f"{w.name} backward: {w.description}", flops_per_step=flops,
+                       l2=f"inputs {6 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2; no flush"),
         "roofline": {
             "bound": "tensor",
             "achieved": round(achieved, 2),
@@ -577,7 +644,9 @@ def bench_ours_bwd(args):
         "device_error": err,
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_bwd(inp, hdo, budget_s=args.cpu_budget)
+        cb = cpu_baseline_bwd(inp, hdo, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {key: cb[key] for key in ("value", "unit", "cores", "kind",
+                                                         "sample")}
     return line
 
 
@@ -604,7 +673,19 @@ def bench_reference(args):
         sample(budget)
     vals = [sample(budget) for _ in range(args.steps)]
     v = round(statistics.median(x["value"] for x in vals), 6)
+    step_s = [x["seconds"] for x in vals]
+    n_prob = [x["problems"] for x in vals]
     flops = (2.5 if bwd else 1.0) * workloads.flops(inp["lengths"], H, d, True)
+    cfg = workload_config(w, inp, world)
+    if bwd:
+        cfg["workload"] = f"{w.name} backward: {w.description}"
+        cfg["flops_per_step"] = flops
+        cfg["l2"] = f"inputs {6 * T * H * d * 2 / 1e6:.0f} MB > 126 MB L2; no flush"
+    n_all = len(inp["lengths"]) * H
+    sample_desc = (f"each step: whole (document, head) problems, largest documents first, "
+                   f"until {budget:.1f} s of fp64 {'gradient ' if bwd else ''}oracle work "
+                   f"({min(n_prob)}-{max(n_prob)} of {n_all} problems); value = FLOPs done / "
+                   f"time, median over steps")
     return {
         "impl": "reference",
         "metric": METRIC_BWD if bwd else METRIC,
@@ -613,18 +694,19 @@ def bench_reference(args):
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(flops / (v * 1e12) * 1e3, 3) if v else None,
+        "ms_per_step": round(1e3 * statistics.mean(step_s), 1),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16, see workloads.py)",
-        "config": {"workload": f"{w.name}: {w.description}", "tokens": T, "heads": H,
-                   "head_dim": d, "causal": True, "flops_per_step": flops},
+        "config": cfg,
         "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": vals[0]["cores"],
-                         "kind": "oracle", "sample": vals[0]["sample"] + " per step"},
+                         "kind": "oracle", "sample": sample_desc},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
+        "note": "ms_per_step is the host time of one timed sample step, not of the whole "
+                "workload",
     }
 
 
@@ -637,6 +719,9 @@ def main():
     ap.add_argument("--workload", default="dense_causal", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="time only --workload (default: dense_causal plus the packed, "
+                         "long-context and MXFP8 workloads as a `workloads` sub-object)")
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"])
     args = ap.parse_args()
     if args.warmup < 3:

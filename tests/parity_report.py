@@ -4,9 +4,8 @@
 
 Runs every configuration through the C ABI and compares with the fp64 oracle
 the way the GPU tests do: the tiny config element by element (causal and
-non-causal), the large ones on sampled rows (384 random rows plus every
-document's first, second, 128th, 129th, 256th, 257th and last row, random
-heads), MXFP8 against the oracle on the exactly dequantised inputs.  Prints
+non-causal), the large ones too (every (document, head) problem in a spawned
+process pool), MXFP8 against the oracle on the exactly dequantised inputs.  Prints
 max / mean absolute output error, max absolute lse error and the tolerance
 each is held to.  Then the backward on the GPU tests' cases, every element of
 dq, dk, dv against the fp64 gradient oracle, errors relative to each
@@ -28,24 +27,11 @@ sys.path.insert(0, HERE)
 
 from exact_tiled_attention_39_b200 import attn as A  # noqa: E402
 from exact_tiled_attention_39_b200 import workloads  # noqa: E402
-from oracle.attention import ref_attention, ref_attention_rows  # noqa: E402
+from oracle.attention import ref_attention  # noqa: E402
 from oracle.attention_bwd import ref_attention_bwd  # noqa: E402
 from oracle.mxfp8 import dequantize_mxfp8_ref, quantize_mxfp8_ref  # noqa: E402
 from helpers import BF16_MAX_ABS, BF16_MEAN_ABS, LSE_ABS, MXFP8_MAX_ABS, run_gpu  # noqa: E402
-
-
-def sample_rows(lengths, H, n, seed):
-    rng = np.random.default_rng(seed)
-    starts = np.concatenate([[0], np.cumsum(lengths)])
-    toks = set(rng.integers(0, int(starts[-1]), n).tolist())
-    for a, b in zip(starts[:-1], starts[1:]):
-        for off in (0, 1, 127, 128, 255, 256):
-            if a + off < b:
-                toks.add(int(a + off))
-        if b > a:
-            toks.add(int(b - 1))
-    toks = np.array(sorted(toks))
-    return toks, rng.integers(0, H, len(toks))
+from oracle_pool import full_reference  # noqa: E402
 
 
 def deq(x):
@@ -129,16 +115,15 @@ def main():
         out, lse, _ = run_gpu(inp["q"], inp["k"], inp["v"], cu, True, inp["scale"],
                               dtype=A.ATTN_MXFP8 if fp8 else A.ATTN_BF16,
                               max_seqlen=max(inp["lengths"]))
-        toks, heads = sample_rows(inp["lengths"], inp["q"].shape[1], 384, seed=1)
         if fp8:
             q, k, v = deq(inp["q"]), deq(inp["k"]), deq(inp["v"])
         else:
             q, k, v = (inp[n].double().numpy() for n in ("q", "k", "v"))
-        ro, rl = ref_attention_rows(q, k, v, cu.numpy(), True, inp["scale"], toks, heads)
-        e = np.abs(out[toks, heads].double().numpy() - ro)
-        le = np.abs(lse[heads, toks].double().numpy() - rl)
-        out_lines.append(line(name, len(toks), e, le, MXFP8_MAX_ABS if fp8 else BF16_MAX_ABS,
-                              None if fp8 else BF16_MEAN_ABS))
+        ro, rl = full_reference(q, k, v, inp["lengths"], True, inp["scale"])
+        e = np.abs(out.double().numpy() - ro)
+        le = np.abs(lse.double().numpy() - rl)
+        out_lines.append(line(name, ro.shape[0] * ro.shape[1], e, le,
+                              MXFP8_MAX_ABS if fp8 else BF16_MAX_ABS, BF16_MEAN_ABS))
     out_lines += bwd_lines()
     for l_ in out_lines:
         print(json.dumps(l_))

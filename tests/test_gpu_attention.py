@@ -13,6 +13,7 @@ from exact_tiled_attention_39_b200 import build, workloads
 from oracle.attention import ref_attention, ref_attention_rows, visible_count
 from oracle.schedule import schedule_ref
 from helpers import (BF16_MAX_ABS, BF16_MEAN_ABS, LSE_ABS, errors, run_gpu)
+from oracle_pool import full_reference
 
 pytestmark = pytest.mark.gpu
 
@@ -226,7 +227,26 @@ def _sample_rows(lengths, H, n, seed):
 
 
 @pytest.mark.parametrize("name", ["dense_causal", "packed_causal", "long_outlier"])
-def test_full_workload(name):
+def test_full_workload_every_element(name):
+    """The full-size workloads in the launch configuration bench.py times,
+    compared with the fp64 oracle on every element of out and lse (every
+    (document, head) problem, computed in a spawned process pool)."""
+    inp = workloads.make_inputs(name)
+    cu = inp["cu_seqlens"]
+    out, lse, ws = run_gpu(inp["q"], inp["k"], inp["v"], cu, True, inp["scale"],
+                           max_seqlen=max(inp["lengths"]))
+    assert A.attn_get_device_error(ws) == 0
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    ro, rl = full_reference(inp["q"].double().numpy(), inp["k"].double().numpy(),
+                            inp["v"].double().numpy(), inp["lengths"], True, inp["scale"])
+    mx, mean, le = errors(out, lse, ro, rl)
+    assert mx <= BF16_MAX_ABS and mean <= BF16_MEAN_ABS and le <= LSE_ABS, (mx, mean, le)
+
+
+@pytest.mark.parametrize("name", ["dense_causal", "packed_causal"])
+def test_full_workload_sampled_rows(name):
+    """Fast path of the check above: sampled rows (every document's edges and
+    tile edges plus random rows), each computed on its own by the oracle."""
     inp = workloads.make_inputs(name)
     w = inp["workload"]
     cu = inp["cu_seqlens"]
@@ -237,17 +257,9 @@ def test_full_workload(name):
     ro, rl = ref_attention_rows(inp["q"].double().numpy(), inp["k"].double().numpy(),
                                 inp["v"].double().numpy(), cu.numpy(), True, inp["scale"],
                                 toks, heads)
-    o = out[toks, heads].double().numpy()
-    e = np.abs(o - ro)
+    e = np.abs(out[toks, heads].double().numpy() - ro)
     assert e.max() <= BF16_MAX_ABS and e.mean() <= BF16_MEAN_ABS, (e.max(), e.mean())
     assert np.abs(lse[heads, toks].double().numpy() - rl).max() <= LSE_ABS
-    # properties of every row: finite, and each output is a convex combination
-    # of value rows (within bf16 rounding of the result)
-    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
-    vmax = inp["v"].float().amax(dim=0)
-    vmin = inp["v"].float().amin(dim=0)
-    of = out.float()
-    assert (of <= vmax + 0.02 * vmax.abs() + 1e-2).all() and (of >= vmin - 0.02 * vmin.abs() - 1e-2).all()
 
 
 @pytest.mark.parametrize("name", ["packed_causal", "long_outlier"])
