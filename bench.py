@@ -1,7 +1,7 @@
 """Benchmark of the exact tiled attention forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload dense_causal|packed_causal|long_outlier|mxfp8_packed]
+                    [--workload dense_causal|packed_causal|long_outlier|mxfp8_packed|mxfp8_incoherent]
                     [--pass fwd|bwd]
 
 One step = one ``attn_fwd`` call through the C ABI (the schedule-build
@@ -205,7 +205,7 @@ class ClockSampler:
 
 KERNEL_TIMING_LAUNCHES = 50       # per-kernel time: median of at least this many launches
 KERNEL_TIMING_MIN_S = 1.0         # ... and of at least this much device time (clock samples)
-EXTRA_WORKLOADS = ("packed_causal", "long_outlier", "mxfp8_packed")
+EXTRA_WORKLOADS = ("packed_causal", "long_outlier", "mxfp8_packed", "mxfp8_incoherent")
 
 
 def kernel_name_for(dtype_name: str) -> str:
@@ -234,10 +234,16 @@ def measure_workload(A, name, steps, warmup, dev, stream, pg):
     out = torch.empty_like(q)
     lse = torch.empty((H, T), dtype=torch.float32, device=dev)
     ws = A.make_workspace(A.Shape(T, len(lengths), H, d, max_seqlen), dtype, dev)
+    if w.incoherent:
+        signs = inp["signs"].to(dev)
 
-    def step():
-        A.attn_fwd(q, k, v, cu, out, lse, causal, inp["scale"], dtype=dtype, stream=stream,
-                   workspace=ws, max_seqlen=max_seqlen)
+        def step():
+            A.attn_fwd_incoherent(q, k, v, cu, out, lse, causal, inp["scale"], signs,
+                                  stream=stream, workspace=ws, max_seqlen=max_seqlen)
+    else:
+        def step():
+            A.attn_fwd(q, k, v, cu, out, lse, causal, inp["scale"], dtype=dtype, stream=stream,
+                       workspace=ws, max_seqlen=max_seqlen)
 
     for _ in range(warmup):
         step()
@@ -447,6 +453,7 @@ def cpu_baseline(w, inp, budget_s=15.0):
     """Time the fp64 oracle on the host cores on a bounded sample of the
     workload: whole (document, head) problems, as many as fit the budget."""
     from oracle.attention import ref_attention
+    from oracle.incoherent import incoherent_operands
     from oracle.mxfp8 import quantize_mxfp8_ref, dequantize_mxfp8_ref
 
     cores = len(os.sched_getaffinity(0))
@@ -463,9 +470,12 @@ def cpu_baseline(w, inp, budget_s=15.0):
         q = inp["q"][a:b, h:h + 1].double().numpy()
         k = inp["k"][a:b, h:h + 1].double().numpy()
         v = inp["v"][a:b, h:h + 1].double().numpy()
-        if w.dtype == "mxfp8":
+        scale = inp["scale"]
+        if w.incoherent:
+            q, k, v, scale = incoherent_operands(q, k, v, scale, inp["signs"].numpy())
+        elif w.dtype == "mxfp8":
             q, k, v = (dequantize_mxfp8_ref(*quantize_mxfp8_ref(x)) for x in (q, k, v))
-        ref_attention(q, k, v, [0, b - a], True, inp["scale"])
+        ref_attention(q, k, v, [0, b - a], True, scale)
         done_flops += workloads.flops([b - a], 1, d, True)
         done += 1
         if time.perf_counter() - t_start > budget_s:

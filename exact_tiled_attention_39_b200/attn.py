@@ -15,8 +15,8 @@ import torch
 __all__ = ["ATTN_BF16", "ATTN_MXFP8", "AttnError", "lib", "workspace_size", "attn_fwd",
            "attn_fwd_noalloc", "attn_quantize_mxfp8", "attn_get_device_error", "status_string",
            "make_workspace", "attn_timing_enable", "attn_timing_read", "bwd_workspace_size",
-           "make_bwd_workspace", "attn_bwd", "attn_quantize_mxfp8_rotated", "LIB_PATH",
-           "EXPORTED_SYMBOLS"]
+           "make_bwd_workspace", "attn_bwd", "attn_quantize_mxfp8_rotated",
+           "attn_fwd_incoherent", "LIB_PATH", "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 
@@ -31,7 +31,8 @@ STATUS = {
 EXPORTED_SYMBOLS = ("attn_workspace_size", "attn_fwd", "attn_quantize_mxfp8",
                     "attn_get_device_error", "attn_status_string", "attn_abi_version",
                     "attn_fwd_noalloc", "attn_timing_enable", "attn_timing_read",
-                    "attn_bwd_workspace_size", "attn_bwd", "attn_quantize_mxfp8_rotated")
+                    "attn_bwd_workspace_size", "attn_bwd", "attn_quantize_mxfp8_rotated",
+                    "attn_fwd_incoherent")
 
 
 class AttnError(RuntimeError):
@@ -82,6 +83,9 @@ def lib() -> ctypes.CDLL:
         L.attn_bwd.restype = ctypes.c_int
         L.attn_quantize_mxfp8_rotated.argtypes = [vp, vp, vp, vp, i64, i32, vp]
         L.attn_quantize_mxfp8_rotated.restype = ctypes.c_int
+        L.attn_fwd_incoherent.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_float,
+                                          vp, vp, ctypes.POINTER(_Shape), vp, sz]
+        L.attn_fwd_incoherent.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -147,6 +151,32 @@ def attn_fwd(q, k, v, cu_seqlens, out, lse, causal: bool, scale: float, dtype: i
                             workspace.numel())
     if rc != 0:
         raise AttnError(rc, "attn_fwd")
+    return workspace
+
+
+def attn_fwd_incoherent(q, k, v, cu_seqlens, out, lse, causal: bool, scale: float, signs,
+                        stream=None, workspace=None, max_seqlen: int | None = None,
+                        num_seqs: int | None = None):
+    """The MXFP8 forward with incoherent processing (``attn_fwd_incoherent``):
+    Q and K rotated by diag(signs) H_d before quantisation, the softmax scale
+    divided by d inside the call.  signs: fp32 [d] of +-1 on q's device.
+    Other arguments as ``attn_fwd``; the workspace is the MXFP8 one."""
+    shape = _check_fwd_args(q, k, v, out, lse, cu_seqlens, max_seqlen, num_seqs)
+    if (signs.dtype != torch.float32 or not signs.is_cuda or not signs.is_contiguous()
+            or tuple(signs.shape) != (q.shape[2],) or signs.device != q.device):
+        raise ValueError(f"signs must be a contiguous fp32 tensor of shape [d] on {q.device}")
+    with torch.cuda.device(q.device):
+        if workspace is None:
+            workspace = make_workspace(shape, ATTN_MXFP8, q.device)
+        elif not workspace.is_cuda or workspace.device != q.device:
+            raise ValueError("workspace must be on the same CUDA device as q")
+        s = shape.c()
+        rc = lib().attn_fwd_incoherent(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(out),
+                                       _ptr(lse), int(bool(causal)), float(scale), _ptr(signs),
+                                       _stream_handle(stream, q.device), ctypes.byref(s),
+                                       _ptr(workspace), workspace.numel())
+    if rc != 0:
+        raise AttnError(rc, "attn_fwd_incoherent")
     return workspace
 
 

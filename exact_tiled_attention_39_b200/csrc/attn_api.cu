@@ -12,6 +12,7 @@
 #include "attn_fwd_pair_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
 #include "common.cuh"
+#include "incoherent.cuh"
 #include "quant_mxfp8.cuh"
 #include "schedule.cuh"
 
@@ -219,10 +220,18 @@ attn_status_t attn_quantize_mxfp8(const void* x, uint8_t* codes, uint8_t* scales
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+}  // extern "C"
+
+namespace attn {
+namespace {
+
+// The forward of attn_fwd and attn_fwd_incoherent.  signs != nullptr (MXFP8
+// only) selects incoherent processing: Q and K rotated by diag(signs) H_d
+// in the pre-pass, the softmax scale divided by d.
+attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
                        void* out, float* lse, int causal, float scale, attn_dtype_t dtype,
-                       void* stream, const attn_shape_t* shape, void* workspace,
-                       size_t workspace_bytes) {
+                       const float* signs, void* stream, const attn_shape_t* shape,
+                       void* workspace, size_t workspace_bytes) {
   const attn_status_t st = check_shape(shape);
   if (st != ATTN_OK) return st;
   if (dtype != ATTN_BF16 && dtype != ATTN_MXFP8) return ATTN_ERR_UNSUPPORTED;
@@ -266,7 +275,35 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   // the E4M3 codes of q and k, and P V on the exact bf16 dequantisation of v;
   // with d = 64 all three products run on the dequantised values.
   const void* qk_src[2] = {q, k};
-  if (dtype == ATTN_MXFP8) {
+  if (dtype == ATTN_MXFP8 && signs != nullptr) {
+    // Incoherent processing: one launch for the three tensors, one thread per
+    // (token, head) row; Q and K rotated, V quantised as it is.  Outputs as
+    // for the plain pre-pass below.
+    RowQuantJobs jobs;
+    jobs.rows = static_cast<long long>(s.total_tokens) * s.num_heads;
+    const void* src[3] = {q, k, v};
+    for (int i = 0; i < 3; ++i) {
+      const bool use_codes = fp8_kernel && i < 2;
+      jobs.t[i].x = static_cast<const uint4*>(src[i]);
+      jobs.t[i].codes = use_codes ? reinterpret_cast<uint4*>(ws + wl.codes_off[i]) : nullptr;
+      jobs.t[i].scales = use_codes ? ws + wl.scales_off[i] : nullptr;
+      jobs.t[i].deq = use_codes ? nullptr : reinterpret_cast<uint4*>(ws + wl.deq_off[i]);
+      jobs.t[i].rotate = i < 2 ? 1 : 0;
+    }
+    const long long qgrid = (jobs.rows + 127) / 128;
+    if (qgrid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    if (s.head_dim == 128)
+      quantize_mxfp8_incoherent_qkv_kernel<128>
+          <<<dim3(static_cast<unsigned>(qgrid), 3), 128, 0, strm>>>(jobs, signs);
+    else
+      quantize_mxfp8_incoherent_qkv_kernel<64>
+          <<<dim3(static_cast<unsigned>(qgrid), 3), 128, 0, strm>>>(jobs, signs);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    for (int i = 0; i < 2; ++i) qk_src[i] = ws + (fp8_kernel ? wl.codes_off[i] : wl.deq_off[i]);
+    v = ws + wl.deq_off[2];
+    // (Q M)(K M)^T = d Q K^T: exact division by the power of two d
+    scale /= static_cast<float>(s.head_dim);
+  } else if (dtype == ATTN_MXFP8) {
     // One launch for all three tensors.  The block-scaled kernel reads the
     // codes and scales of Q and K and the exact dequantised V; the head-dim
     // 64 fallback reads dequantised Q, K and V.
@@ -339,6 +376,32 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
   }
   timing_mark(2, strm);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace attn
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                       void* out, float* lse, int causal, float scale, attn_dtype_t dtype,
+                       void* stream, const attn_shape_t* shape, void* workspace,
+                       size_t workspace_bytes) {
+  return fwd_impl(q, k, v, cu_seqlens, out, lse, causal, scale, dtype, nullptr, stream, shape,
+                  workspace, workspace_bytes);
+}
+
+attn_status_t attn_fwd_incoherent(const void* q, const void* k, const void* v,
+                                  const int32_t* cu_seqlens, void* out, float* lse, int causal,
+                                  float scale, const float* signs, void* stream,
+                                  const attn_shape_t* shape, void* workspace,
+                                  size_t workspace_bytes) {
+  if (shape != nullptr && shape->total_tokens > 0) {
+    if (signs == nullptr) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(signs) & 3u) != 0) return ATTN_ERR_ALIGNMENT;
+  }
+  return fwd_impl(q, k, v, cu_seqlens, out, lse, causal, scale, ATTN_MXFP8,
+                  signs != nullptr ? signs : nullptr, stream, shape, workspace, workspace_bytes);
 }
 
 attn_status_t attn_timing_enable(int32_t enable) {
@@ -602,7 +665,6 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
 // Incoherent processing: attn_quantize_mxfp8_rotated.  The forward's and the
 // backward's sources end above this line.
 // ===========================================================================
-#include "incoherent.cuh"
 
 extern "C" attn_status_t attn_quantize_mxfp8_rotated(const void* x, const float* signs,
                                                      uint8_t* codes, uint8_t* scales,

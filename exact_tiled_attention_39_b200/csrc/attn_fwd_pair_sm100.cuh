@@ -44,6 +44,11 @@ namespace attn {
 #endif
 constexpr bool kFaultDropFirstScoreCommit = ATTN_FAULT_DROP_FIRST_SCORE_COMMIT != 0;
 
+#ifndef ATTN_PINGPONG
+#define ATTN_PINGPONG 1
+#endif
+constexpr bool kPingPong = ATTN_PINGPONG != 0;
+
 constexpr int kPairThreads = 512;
 constexpr uint32_t kPairRegsSoftmax = 184, kPairRegsEpilogue = 64, kPairRegsOther = 80;
 static_assert(2 * kPairRegsSoftmax + kPairRegsEpilogue + kPairRegsOther == 4 * 128,
@@ -72,7 +77,8 @@ struct PairLayout {
   static constexpr int kOEmpty = kOUnit + 2;                  // + tile
   static constexpr int kStFull = kOEmpty + 2;                 // + tile
   static constexpr int kStEmpty = kStFull + 2;                // + tile
-  static constexpr int kDrain = kStEmpty + 2;
+  static constexpr int kTok = kStEmpty + 2;                   // + 2 * warp pair + tile
+  static constexpr int kDrain = kTok + 8;
   static constexpr int kUnitFull = kDrain + 1;                // + slot
   static constexpr int kUnitEmpty = kUnitFull + kUnitSlots;   // + slot
   static constexpr int kNumBars = kUnitEmpty + kUnitSlots;
@@ -129,6 +135,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       ptx::mbar_init(bar(Lay::kStFull + t), 4);
       ptx::mbar_init(bar(Lay::kStEmpty + t), 4);
     }
+    for (int i = 0; i < 8; ++i) ptx::mbar_init(bar(Lay::kTok + i), 1);
     ptx::mbar_init(bar(Lay::kDrain), 1);
     for (int i = 0; i < kUnitSlots; ++i) {
       ptx::mbar_init(bar(Lay::kUnitFull + i), 1);
@@ -179,6 +186,27 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const float c = p.scale_log2;
     const uint64_t c2 = ptx::f2_pack(c, c);
     uint32_t g = 0, st_cnt = 0;                    // this tile's key steps, units handed over
+    // Exponential phases of the two tiles take turns on each SM
+    // sub-partition: warp w of tile A and warp w of tile B share one, and a
+    // token passed between them (an mbarrier each way) lets only one of
+    // them run its exponentials at a time.  Tile A goes first.  Both warps
+    // take the same number of turns per unit (the larger step count of the
+    // two tiles; a tile with fewer steps passes the token on unused).
+    const int pair = warp & 3;
+    const uint32_t tok_mine = bar(Lay::kTok + 2 * pair + t);
+    const uint32_t tok_other = bar(Lay::kTok + 2 * pair + (1 - t));
+    uint32_t turns = 0;
+    auto take_turn = [&]() -> bool {
+      if (!kPingPong) return true;
+      const bool r2 = wait_warp(tok_mine, (turns & 1) ^ (t == 0 ? 1u : 0u), ctl);
+      ++turns;
+      return r2;
+    };
+    auto pass_turn = [&]() {
+      if (!kPingPong) return;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(tok_other);
+    };
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
       const int4 uw = next_unit_warp(k, ok);
@@ -186,7 +214,12 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const int doc_len = uw.y;
       const int qb = 2 * uw.z + t;
       const int n = tile_steps(qb, doc_len, causal);
-      if (n == 0) continue;
+      const int n_turns = max(n, tile_steps(2 * uw.z + (1 - t), doc_len, causal));
+      if (n == 0) {
+        for (int j = 0; j < n_turns && ok; ++j)
+          if ((ok = take_turn())) pass_turn();
+        continue;
+      }
       float m_used = -INFINITY;   // running maximum in log2 units
       float l = 0.f;              // sum of the weights
       float l_round = 0.f;        // sum of the weights as rounded to bf16
@@ -195,13 +228,10 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::tc_fence_after();
         float s[128];
         {
-          uint32_t sa[64];
-          ptx::tmem_ld_x64(t_s, sa);
+          uint32_t sa[128];
+          ptx::tmem_ld_2x64(t_s, sa);
 #pragma unroll
-          for (int q = 0; q < 64; ++q) s[q] = __uint_as_float(sa[q]);
-          ptx::tmem_ld_x64(t_s + 64, sa);
-#pragma unroll
-          for (int q = 0; q < 64; ++q) s[64 + q] = __uint_as_float(sa[q]);
+          for (int q = 0; q < 128; ++q) s[q] = __uint_as_float(sa[q]);
         }
         const bool diag = causal && j == qb;
         if (diag || (j + 1) * kBlockN > doc_len) {
@@ -245,6 +275,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         // Weights rounded to bf16 for the P V product; O is divided by the
         // sum of the rounded weights, the log-sum-exp uses the exact sum.
+        if (!(ok = take_turn())) break;
         {
           const float base = m_used == -INFINITY ? 0.f : m_used;
           const uint64_t nb2 = ptx::f2_pack(-base, -base);
@@ -282,11 +313,15 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           l += e0 + e1;
           l_round += (sr[0] + sr[1]) + (sr[2] + sr[3]);
         }
+        pass_turn();
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(bar(Lay::kPFull + t));
       }
+      if (!ok) break;
+      for (int j = n; j < n_turns && ok; ++j)
+        if ((ok = take_turn())) pass_turn();
       if (!ok) break;
       if (!(ok = wait_warp(bar(Lay::kStEmpty + t), (st_cnt & 1) ^ 1, ctl))) break;
       ++st_cnt;

@@ -42,6 +42,89 @@ __device__ __forceinline__ uint32_t quantize_block_f32(const float* v, uint32_t 
   return code;
 }
 
+// The rows of one tensor for the incoherent pre-pass of an attention call:
+// any of codes, scales and deq may be null (not written).
+struct RowQuantJob {
+  const uint4* x;       // bf16 [rows][D]
+  uint4* codes;         // E4M3 [rows][D]
+  uint8_t* scales;      // E8M0 [rows][D / 32]
+  uint4* deq;           // bf16 [rows][D]: exact dequantised values
+  int rotate;           // 1: (x * s) H_d before quantisation; 0: x as it is
+};
+struct RowQuantJobs {
+  RowQuantJob t[3];
+  long long rows;       // per tensor
+};
+
+// One row: load, optionally rotate, quantise each 32-element block and write
+// what the job asks for.
+template <int D>
+__device__ __forceinline__ void quantize_row(const RowQuantJob& j, const float* __restrict__ signs,
+                                             long long row) {
+  float y[D];
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) {
+    const uint4 w = j.x[row * (D / 8) + i];
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      y[8 * i + 2 * q] = bf16_lo(ws[q]);
+      y[8 * i + 2 * q + 1] = bf16_hi(ws[q]);
+    }
+  }
+  if (j.rotate) {
+#pragma unroll
+    for (int i = 0; i < D; ++i) y[i] *= signs[i];          // exact: +-1
+#pragma unroll
+    for (int h = 1; h < D; h <<= 1) {
+#pragma unroll
+      for (int b0 = 0; b0 < D; b0 += 2 * h) {
+#pragma unroll
+        for (int q = 0; q < h; ++q) {
+          const float a = y[b0 + q], b = y[b0 + q + h];
+          y[b0 + q] = __fadd_rn(a, b);
+          y[b0 + q + h] = __fsub_rn(a, b);
+        }
+      }
+    }
+  }
+  uint32_t sc = 0;
+#pragma unroll
+  for (int blk = 0; blk < D / 32; ++blk) {
+    uint32_t out[8];
+    const uint32_t code = quantize_block_f32(y + 32 * blk, out);
+    sc |= code << (8 * blk);
+    if (j.codes != nullptr) {
+      j.codes[row * (D / 16) + 2 * blk] = make_uint4(out[0], out[1], out[2], out[3]);
+      j.codes[row * (D / 16) + 2 * blk + 1] = make_uint4(out[4], out[5], out[6], out[7]);
+    }
+    if (j.deq != nullptr) {
+      // E4M3 value * 2^(code - 127): exact in bf16 (code 0 needs 2^-127)
+      const float mul = code == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(code << 23);
+      uint32_t o[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float f0, f1, f2, f3;
+        e4m3x2_to_f32(static_cast<uint16_t>(out[i] & 0xFFFFu), f0, f1);
+        e4m3x2_to_f32(static_cast<uint16_t>(out[i] >> 16), f2, f3);
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[2 * i]) : "f"(f1 * mul), "f"(f0 * mul));
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(o[2 * i + 1]) : "f"(f3 * mul), "f"(f2 * mul));
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        j.deq[row * (D / 8) + 4 * blk + i] =
+            make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+    }
+  }
+  if (j.scales != nullptr) {
+    if (D == 128) {
+      reinterpret_cast<uint32_t*>(j.scales)[row] = sc;
+    } else {
+      reinterpret_cast<uint16_t*>(j.scales)[row] = static_cast<uint16_t>(sc);
+    }
+  }
+}
+
 // One thread per row of D bf16 values: codes [rows][D] (E4M3), scales
 // [rows][D / 32] (E8M0), signs: D fp32 values (+-1).
 template <int D>
@@ -52,43 +135,21 @@ quantize_mxfp8_rotated_kernel(const uint4* __restrict__ x, const float* __restri
   static_assert(D == 64 || D == 128, "head dim 64 or 128");
   const long long row = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (row >= rows) return;
-  float y[D];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) {
-    const uint4 w = x[row * (D / 8) + i];
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      y[8 * i + 2 * j] = bf16_lo(ws[j]) * signs[8 * i + 2 * j];          // exact: +-1
-      y[8 * i + 2 * j + 1] = bf16_hi(ws[j]) * signs[8 * i + 2 * j + 1];
-    }
-  }
-#pragma unroll
-  for (int h = 1; h < D; h <<= 1) {
-#pragma unroll
-    for (int b0 = 0; b0 < D; b0 += 2 * h) {
-#pragma unroll
-      for (int j = 0; j < h; ++j) {
-        const float a = y[b0 + j], b = y[b0 + j + h];
-        y[b0 + j] = __fadd_rn(a, b);
-        y[b0 + j + h] = __fsub_rn(a, b);
-      }
-    }
-  }
-  uint32_t sc = 0;
-#pragma unroll
-  for (int blk = 0; blk < D / 32; ++blk) {
-    uint32_t out[8];
-    const uint32_t code = quantize_block_f32(y + 32 * blk, out);
-    sc |= code << (8 * blk);
-    codes[row * (D / 16) + 2 * blk] = make_uint4(out[0], out[1], out[2], out[3]);
-    codes[row * (D / 16) + 2 * blk + 1] = make_uint4(out[4], out[5], out[6], out[7]);
-  }
-  if (D == 128) {
-    reinterpret_cast<uint32_t*>(scales)[row] = sc;
-  } else {
-    reinterpret_cast<uint16_t*>(scales)[row] = static_cast<uint16_t>(sc);
-  }
+  const RowQuantJob j{x, codes, scales, nullptr, 1};
+  quantize_row<D>(j, signs, row);
+}
+
+// The pre-pass of an attention call with incoherent processing: Q and K
+// rotated then quantised, V quantised as it is, all three in one launch
+// (blockIdx.y picks the tensor).
+template <int D>
+__global__ void __launch_bounds__(128)
+quantize_mxfp8_incoherent_qkv_kernel(const __grid_constant__ RowQuantJobs jobs,
+                                     const float* __restrict__ signs) {
+  static_assert(D == 64 || D == 128, "head dim 64 or 128");
+  const long long row = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (row >= jobs.rows) return;
+  quantize_row<D>(jobs.t[blockIdx.y], signs, row);
 }
 
 }  // namespace attn

@@ -23,7 +23,7 @@ from dataclasses import dataclass, field
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "get", "make_inputs", "draw_doc_lengths",
-           "cu_from_lengths", "tensor_sha256", "flops"]
+           "cu_from_lengths", "tensor_sha256", "flops", "draw_signs"]
 
 
 @dataclass(frozen=True)
@@ -41,6 +41,7 @@ class Workload:
     outlier_channels: tuple[int, ...] = ()
     outlier_factor: float = 1.0
     dtype: str = "bf16"
+    incoherent: bool = False      # MXFP8 with Q, K rotated by random signs + Hadamard
     description: str = ""
     extras: dict = field(default_factory=dict)
 
@@ -70,6 +71,13 @@ WORKLOADS = {
         outlier_channels=(5, 70), outlier_factor=20.0, dtype="mxfp8",
         description="packed as packed_causal (seed 4) with the outlier "
                     "channels of long_outlier, MXFP8"),
+    "mxfp8_incoherent": Workload(
+        name="mxfp8_incoherent", seed=4, heads=32, head_dim=128, causal=(True,),
+        pack_tokens=16384, doc_len_range=(128, 4096),
+        outlier_channels=(5, 70), outlier_factor=20.0, dtype="mxfp8", incoherent=True,
+        description="the mxfp8_packed inputs with incoherent processing (Q, K "
+                    "rotated by random signs and a Hadamard matrix before "
+                    "quantisation; signs from seed 1004)"),
 }
 
 
@@ -128,7 +136,16 @@ def make_inputs(w: Workload | str, heads: int | None = None,
     out["tokens"] = T
     out["scale"] = float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32).item())
     out["workload"] = w
+    if w.incoherent:
+        out["signs"] = draw_signs(1000 + w.seed, d)
     return out
+
+
+def draw_signs(seed: int, d: int) -> torch.Tensor:
+    """d random signs (+1 / -1, fp32) from their own seeded generator: the
+    random draw incoherent processing takes as an input."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    return torch.where(torch.rand(d, generator=g) < 0.5, -1.0, 1.0).to(torch.float32)
 
 
 def tensor_sha256(t: torch.Tensor) -> str:

@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define ATTN_ABI_VERSION 3
+#define ATTN_ABI_VERSION 4
 
 typedef enum {
   ATTN_BF16 = 0,  /* bf16 operands, bf16 tensor-core products, fp32 softmax   */
@@ -112,6 +112,28 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, const int32_
                        void* out, float* lse, int causal, float scale, attn_dtype_t dtype,
                        void* stream, const attn_shape_t* shape, void* workspace,
                        size_t workspace_bytes);
+
+/* The MXFP8 forward with incoherent processing ("FlashAttention, pelatihan
+ * multi-GPU, dan kuantisasi bobot", section 1: FlashAttention-3 multiplies
+ * Q and K by a random orthogonal matrix before FP8 quantisation, spreading
+ * outlier channels over the head dimension; the scores are unchanged in
+ * exact arithmetic).  Same arguments as attn_fwd with dtype ATTN_MXFP8,
+ * plus signs: device fp32 [head_dim], each +1 or -1 (the caller's random
+ * draw), 4-byte aligned, required when total_tokens > 0 (else
+ * ATTN_ERR_INVALID_ARG).  Each row of q and k (one token of one head)
+ * becomes (x * signs) H_d in fp32 (H_d the unnormalised Sylvester Hadamard
+ * matrix, computed by the butterfly described at attn_quantize_mxfp8_rotated)
+ * and is then quantised as by attn_quantize_mxfp8; v is quantised as it is;
+ * the attention runs as for ATTN_MXFP8 with the softmax scale divided by
+ * head_dim (the rotation multiplies every score by head_dim).  out and lse
+ * are in the units of the unrotated problem.  Workspace: attn_workspace_size
+ * of the shape with ATTN_MXFP8.  Launches the schedule-build kernel, one
+ * rotating quantisation kernel for q, k and v, and the attention kernel. */
+attn_status_t attn_fwd_incoherent(const void* q, const void* k, const void* v,
+                                  const int32_t* cu_seqlens, void* out, float* lse, int causal,
+                                  float scale, const float* signs, void* stream,
+                                  const attn_shape_t* shape, void* workspace,
+                                  size_t workspace_bytes);
 
 /* attn_fwd for callers that cannot allocate device memory: a plugin or
  * custom operator that its host application hands only input and output

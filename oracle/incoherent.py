@@ -33,7 +33,7 @@ from .attention import ref_attention
 from .mxfp8 import dequantize_mxfp8_ref, quantize_mxfp8_ref
 
 __all__ = ["hadamard", "incoherent_matrix", "rotate_fp64", "rotate_fp32",
-           "ref_attention_incoherent_mxfp8"]
+           "incoherent_operands", "ref_attention_incoherent_mxfp8"]
 
 
 def hadamard(d: int) -> np.ndarray:
@@ -74,13 +74,21 @@ def rotate_fp32(x, signs) -> np.ndarray:
     return y
 
 
-def ref_attention_incoherent_mxfp8(q, k, v, cu_seqlens, causal: bool, scale: float, signs):
-    """Attention on MXFP8 operands with incoherent processing: Q and K
-    rotated (fp32, as above), the three operands quantised and exactly
-    dequantised by the oracle quantiser, then the fp64 attention with the
-    softmax scale divided by d.  Returns (out, lse) like ``ref_attention``."""
+def incoherent_operands(q, k, v, scale: float, signs):
+    """The operands the attention sees under incoherent processing: Q and K
+    rotated (fp32, as above), the three quantised and exactly dequantised by
+    the oracle quantiser, and the softmax scale divided by d.  Returns
+    (qd, kd, vd, scale / d)."""
     d = np.asarray(q).shape[-1]
     qd = dequantize_mxfp8_ref(*quantize_mxfp8_ref(rotate_fp32(q, signs)))
     kd = dequantize_mxfp8_ref(*quantize_mxfp8_ref(rotate_fp32(k, signs)))
     vd = dequantize_mxfp8_ref(*quantize_mxfp8_ref(np.asarray(v, dtype=np.float64)))
-    return ref_attention(qd, kd, vd, cu_seqlens, causal, scale / d)
+    return qd, kd, vd, scale / d
+
+
+def ref_attention_incoherent_mxfp8(q, k, v, cu_seqlens, causal: bool, scale: float, signs):
+    """Attention on MXFP8 operands with incoherent processing: the fp64
+    attention of ``incoherent_operands``.  Returns (out, lse) like
+    ``ref_attention``."""
+    qd, kd, vd, s = incoherent_operands(q, k, v, scale, signs)
+    return ref_attention(qd, kd, vd, cu_seqlens, causal, s)

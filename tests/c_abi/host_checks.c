@@ -93,6 +93,12 @@ int main(void) {
   check(attn_quantize_mxfp8(NULL, NULL, NULL, 4, 48, NULL) == ATTN_ERR_INVALID_ARG,
         "quantiser: cols not a multiple of 32");
   check(attn_quantize_mxfp8(NULL, NULL, NULL, 0, 64, NULL) == ATTN_OK, "quantiser: empty");
+  check(attn_fwd_incoherent(p16, p16, p16, NULL, p16, (float*)p16, 1, 0.125f, NULL, NULL, &ok,
+                            p16, (size_t)1 << 26) == ATTN_ERR_INVALID_ARG,
+        "incoherent forward: signs required");
+  check(attn_fwd_incoherent(NULL, NULL, NULL, NULL, NULL, NULL, 1, 0.125f, NULL, NULL, &empty,
+                            NULL, 0) == ATTN_OK,
+        "incoherent forward: empty problem is a no-op");
 
   if (failed == 0) printf("c abi host checks: %d ok\n", check_no);
   return failed;

@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_version_and_strings(L):
-    assert L.attn_abi_version() == 3
+    assert L.attn_abi_version() == 4
     assert A.status_string(0) == "ATTN_OK"
     assert A.status_string(5) == "ATTN_ERR_BAD_SEQLENS"
     assert A.status_string(6) == "ATTN_ERR_TIMEOUT"
@@ -148,3 +148,20 @@ def test_rotated_quantiser_host_checks(L):
     assert L.attn_quantize_mxfp8_rotated(vp(16), None, vp(16), vp(16), 4, 128, None) == 1
     assert L.attn_quantize_mxfp8_rotated(vp(16), vp(16), vp(24), vp(16), 4, 64, None) == 3
     assert L.attn_quantize_mxfp8_rotated(vp(16), vp(16), vp(16), vp(18), 4, 64, None) == 3
+
+
+def test_incoherent_forward_host_checks(L):
+    vp = ctypes.c_void_p
+    ok = A.Shape(256, 1, 2, 64, 256).c()
+    empty = A.Shape(0, 0, 2, 64, 0).c()
+    p = vp(16)
+
+    def call(shape, signs, ws_bytes=1 << 26):
+        return L.attn_fwd_incoherent(p, p, p, None, p, p, 1, 0.125, signs, None,
+                                     ctypes.byref(shape) if shape is not None else None, p,
+                                     ws_bytes)
+    assert call(ok, None) == 1                    # signs required
+    assert call(ok, vp(18)) == 3                  # signs misaligned
+    assert call(None, vp(16)) == 1                # no shape
+    assert call(ok, vp(16), ws_bytes=64) == 4     # workspace too small (MXFP8 layout)
+    assert call(empty, None) == 0                 # T == 0: no-op
