@@ -40,7 +40,8 @@ sys.path.insert(0, ROOT)
 from exact_tiled_attention_39_b200 import workloads  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s (causal, bf16 & MXFP8) and % of B200 dense tensor peak"
-METRIC_BWD = "attention bwd TFLOP/s (causal, bf16; 2.5 x forward FLOPs) and % of B200 dense tensor peak"
+METRIC_BWD = ("attention bwd TFLOP/s (causal, bf16 & MXFP8; 2.5 x forward FLOPs) and % of B200 "
+              "dense tensor peak")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -148,28 +149,75 @@ def dist_env():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and throttle-reason samples while the timed kernels run.
+
+    NVML is polled from a background thread about every millisecond (the
+    timed regions last milliseconds, far shorter than nvidia-smi's sampling
+    period); without NVML, nvidia-smi is sampled every 100 ms instead."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device):
+        self.device = device
         self.proc = None
+        self.thread = None
+        self.samples = []       # (sm_mhz, max_mhz, set of reasons)
+        self.source = "none"
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            props = torch.cuda.get_device_properties(self.device)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId_v2(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.device.index or 0)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-        time.sleep(0.25)
+            nv, h = self._nvml_handle()
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            masks = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+            self._stop = threading.Event()
+
+            def poll():
+                while not self._stop.is_set():
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    except Exception:
+                        break
+                    self.samples.append((float(sm), float(mx),
+                                         {n for n, m in masks if rs & m}))
+                    time.sleep(0.001)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            self.source = "nvml, ~1 ms"
+        except Exception:
+            self.thread = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.device.index or 0),
+                     f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms",
+                     "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi, 100 ms"
+                time.sleep(0.25)
+            except OSError:
+                self.proc = None
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             time.sleep(0.15)
             self.proc.terminate()
@@ -178,33 +226,34 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            names = [n for n, _ in self.REASONS]
+            for line in out.splitlines():
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm, mx = float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                self.samples.append((sm, mx, {n for n, v in zip(names, parts[5:9])
+                                              if v.lower() == "active"}))
         return False
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in getattr(self, "lines", []):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [x[0] for x in self.samples]
         loaded = [x for x in sm if x >= 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        reasons = set()
+        for x in self.samples:
+            reasons |= x[2]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": self.samples[-1][1],
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source,
+                "window": "timed steps and the per-kernel timing launches"}
 
 
 KERNEL_TIMING_LAUNCHES = 50       # per-kernel time: median of at least this many launches
-KERNEL_TIMING_MIN_S = 1.0         # ... and of at least this much device time (clock samples)
+KERNEL_TIMING_MIN_S = 0.05        # ... and of at least this much device time
 EXTRA_WORKLOADS = ("packed_causal", "long_outlier", "mxfp8_packed", "mxfp8_incoherent")
 
 
@@ -214,7 +263,7 @@ def kernel_name_for(dtype_name: str) -> str:
     return "attn_fwd_kernel" if dtype_name == "mxfp8" else "attn_fwd_pair_kernel"
 
 
-def measure_workload(A, name, steps, warmup, dev, stream, pg):
+def measure_workload(A, name, steps, warmup, dev, stream, pg, clk):
     """Time one workload: `steps` back-to-back attn_fwd calls (device events,
     barrier + synchronize on both sides, max over ranks), then the attention
     kernel alone (CUDA events the library records on the launching stream
@@ -253,30 +302,30 @@ def measure_workload(A, name, steps, warmup, dev, stream, pg):
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        step()
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
+    with clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        A.attn_timing_enable(True)
+        per, pre = [], []
+        while len(per) < KERNEL_TIMING_LAUNCHES or sum(per) < 1e3 * KERNEL_TIMING_MIN_S:
+            step()
+            a_ms, p_ms = A.attn_timing_read()
+            per.append(a_ms)
+            pre.append(p_ms)
+            if len(per) >= 20000:
+                break
+        A.attn_timing_enable(False)
+        torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
     ms_total = max_over_ranks(pg, t0.elapsed_time(t1), dev)
     ms_step = ms_total / steps
     err = A.attn_get_device_error(ws)
-
-    A.attn_timing_enable(True)
-    per, pre = [], []
-    while len(per) < KERNEL_TIMING_LAUNCHES or sum(per) < 1e3 * KERNEL_TIMING_MIN_S:
-        step()
-        a_ms, p_ms = A.attn_timing_read()
-        per.append(a_ms)
-        pre.append(p_ms)
-        if len(per) >= 20000:
-            break
-    A.attn_timing_enable(False)
-    torch.cuda.synchronize(dev)
     return {
         "w": w, "inp": inp, "dtype": dtype, "flops": flops, "ms_total": ms_total,
         "ms_step": ms_step, "kernel_ms": statistics.median(per),
@@ -324,8 +373,8 @@ def bench_ours(args):
     stream = torch.cuda.current_stream(dev)
     peaks, peak_src = load_peaks()
 
-    with ClockSampler(local) as clk:
-        m = measure_workload(A, args.workload, args.steps, args.warmup, dev, stream, pg)
+    clk = ClockSampler(dev)
+    m = measure_workload(A, args.workload, args.steps, args.warmup, dev, stream, pg, clk)
     w, inp, dtype, flops = m["w"], m["inp"], m["dtype"], m["flops"]
     q, k, v, cu, out, lse = m["tensors"]
     step = m["step"]
@@ -373,8 +422,8 @@ def bench_ours(args):
     extra = {}
     if not args.no_extra_workloads and args.workload == "dense_causal":
         for name in EXTRA_WORKLOADS:
-            with ClockSampler(local) as xclk:
-                mx = measure_workload(A, name, args.steps, args.warmup, dev, stream, pg)
+            xclk = ClockSampler(dev)
+            mx = measure_workload(A, name, args.steps, args.warmup, dev, stream, pg, xclk)
             extra[name] = {
                 "workload": f"{name}: {mx['w'].description}",
                 "dtype": mx["w"].dtype,
@@ -487,10 +536,11 @@ def cpu_baseline(w, inp, budget_s=15.0):
                       f"{el:.1f} s", "seconds": el, "problems": done}
 
 
-def cpu_baseline_bwd(inp, dout, budget_s=15.0):
+def cpu_baseline_bwd(inp, dout, budget_s=15.0, mxfp8=False):
     """The fp64 gradient oracle on the host cores on whole (document, head)
-    problems of the workload, largest documents first, within the budget."""
-    from oracle.attention_bwd import ref_attention_bwd
+    problems of the workload, largest documents first, within the budget
+    (the MXFP8 gradient oracle for an MXFP8 workload)."""
+    from oracle.attention_bwd import ref_attention_bwd, ref_attention_bwd_mxfp8
 
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
@@ -503,7 +553,8 @@ def cpu_baseline_bwd(inp, dout, budget_s=15.0):
     for i, h in problems:
         a, b = int(starts[i]), int(starts[i + 1])
         x = [t[a:b, h:h + 1].double().numpy() for t in (inp["q"], inp["k"], inp["v"], dout)]
-        ref_attention_bwd(*x, [0, b - a], True, inp["scale"])
+        (ref_attention_bwd_mxfp8 if mxfp8 else ref_attention_bwd)(*x, [0, b - a], True,
+                                                                  inp["scale"])
         done_flops += 2.5 * workloads.flops([b - a], 1, d, True)
         done += 1
         if time.perf_counter() - t_start > budget_s:
@@ -524,8 +575,9 @@ def bench_ours_bwd(args):
     pg = init_group("nccl", dev)
 
     w = workloads.get(args.workload)
-    if w.dtype != "bf16":
-        raise SystemExit("--pass bwd: the backward is built for bf16 workloads")
+    if w.incoherent:
+        raise SystemExit("--pass bwd: the backward has no incoherent-processing form")
+    dtype = A.ATTN_MXFP8 if w.dtype == "mxfp8" else A.ATTN_BF16
     inp = workloads.make_inputs(w)
     T, H, d = inp["q"].shape
     causal = True
@@ -541,14 +593,14 @@ def bench_ours_bwd(args):
     out = torch.empty_like(q)
     lse = torch.empty((H, T), dtype=torch.float32, device=dev)
     shape = A.Shape(T, len(lengths), H, d, max_seqlen)
-    A.attn_fwd(q, k, v, cu, out, lse, causal, inp["scale"], max_seqlen=max_seqlen)
+    A.attn_fwd(q, k, v, cu, out, lse, causal, inp["scale"], dtype=dtype, max_seqlen=max_seqlen)
     dq, dk, dv = (torch.empty_like(q) for _ in range(3))
-    ws = A.make_bwd_workspace(shape, dev)
+    ws = A.make_bwd_workspace(shape, dev, dtype)
     stream = torch.cuda.current_stream(dev)
 
     def step():
         A.attn_bwd(q, k, v, out, do, lse, cu, dq, dk, dv, causal, inp["scale"], stream=stream,
-                   workspace=ws, max_seqlen=max_seqlen)
+                   workspace=ws, max_seqlen=max_seqlen, dtype=dtype)
 
     for _ in range(args.warmup):
         step()
@@ -558,7 +610,7 @@ def bench_ours_bwd(args):
     if pg:
         pg.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev) as clk:
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
@@ -625,7 +677,7 @@ def bench_ours_bwd(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "mxfp8" if dtype == A.ATTN_MXFP8 else "bf16",
         "data": "synthetic (seeded N(0,1) bf16, see workloads.py; dout seeded N(0,1))",
         "config": dict(workload_config(w, inp, world),
                        workload=f"{w.name} backward: {w.description}", flops_per_step=flops,
@@ -637,7 +689,8 @@ def bench_ours_bwd(args):
             "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
             "peak_source": f"{peak_source_name(peak_key, 0)} ({peak_src})",
-            "timed_unit": "whole attn_bwd call (4 kernels), device events over the timed steps",
+            "timed_unit": (f"whole attn_bwd call ({5 if dtype == A.ATTN_MXFP8 else 4} kernels), "
+                           "device events over the timed steps"),
             "kernel": "attn_bwd_kernel",
             "traffic": recorded_traffic(w.name, "attn_bwd_kernel", "bwd"),
             "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
@@ -649,12 +702,12 @@ def bench_ours_bwd(args):
             "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
         },
-        "gpu_launches": args.steps * 4,
+        "gpu_launches": args.steps * (5 if dtype == A.ATTN_MXFP8 else 4),
         "clocks": clk.summary(),
         "device_error": err,
     }
     if world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline_bwd(inp, hdo, budget_s=args.cpu_budget)
+        cb = cpu_baseline_bwd(inp, hdo, budget_s=args.cpu_budget, mxfp8=dtype == A.ATTN_MXFP8)
         line["cpu_baseline"] = {key: cb[key] for key in ("value", "unit", "cores", "kind",
                                                          "sample")}
     return line
@@ -674,7 +727,7 @@ def bench_reference(args):
         dout = dout.to(torch.bfloat16)
 
         def sample(budget_s):
-            return cpu_baseline_bwd(inp, dout, budget_s=budget_s)
+            return cpu_baseline_bwd(inp, dout, budget_s=budget_s, mxfp8=w.dtype == "mxfp8")
     else:
         def sample(budget_s):
             return cpu_baseline(w, inp, budget_s=budget_s)

@@ -76,7 +76,7 @@ def lib() -> ctypes.CDLL:
         L.attn_timing_enable.restype = ctypes.c_int
         L.attn_timing_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]
         L.attn_timing_read.restype = ctypes.c_int
-        L.attn_bwd_workspace_size.argtypes = [ctypes.POINTER(_Shape)]
+        L.attn_bwd_workspace_size.argtypes = [ctypes.POINTER(_Shape), ctypes.c_int]
         L.attn_bwd_workspace_size.restype = sz
         L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
                                ctypes.c_float, ctypes.c_int, vp, ctypes.POINTER(_Shape), vp, sz]
@@ -215,13 +215,13 @@ def _doc_shape(q, cu_seqlens, max_seqlen, num_seqs) -> Shape:
     return Shape(T, ns, H, d, int(max_seqlen))
 
 
-def bwd_workspace_size(shape: Shape) -> int:
+def bwd_workspace_size(shape: Shape, dtype: int = ATTN_BF16) -> int:
     s = shape.c()
-    return int(lib().attn_bwd_workspace_size(ctypes.byref(s)))
+    return int(lib().attn_bwd_workspace_size(ctypes.byref(s), dtype))
 
 
-def make_bwd_workspace(shape: Shape, device=None) -> torch.Tensor:
-    n = bwd_workspace_size(shape)
+def make_bwd_workspace(shape: Shape, device=None, dtype: int = ATTN_BF16) -> torch.Tensor:
+    n = bwd_workspace_size(shape, dtype)
     if n == 0:
         raise AttnError(1, "attn_bwd_workspace_size")
     return torch.zeros(n, dtype=torch.uint8, device=device)
@@ -233,7 +233,8 @@ def attn_bwd(q, k, v, out, dout, lse, cu_seqlens, dq, dk, dv, causal: bool, scal
     """Gradients of the forward through the C ABI (``attn_bwd``): q, k, v,
     out (the forward's output), dout: bf16 [T, H, d]; lse: fp32 [H, T] from
     the forward; dq, dk, dv: bf16 [T, H, d], written.  Same document rules
-    as ``attn_fwd``.  Returns the workspace used (allocated if not given)."""
+    as ``attn_fwd``; dtype ATTN_MXFP8 differentiates the MXFP8 forward (out
+    and lse from it).  Returns the workspace used (allocated if not given)."""
     T, H, d = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("dq", dq),
                     ("dk", dk), ("dv", dv)):
@@ -247,7 +248,7 @@ def attn_bwd(q, k, v, out, dout, lse, cu_seqlens, dq, dk, dv, causal: bool, scal
     shape = _doc_shape(q, cu_seqlens, max_seqlen, num_seqs)
     with torch.cuda.device(q.device):
         if workspace is None:
-            workspace = make_bwd_workspace(shape, q.device)
+            workspace = make_bwd_workspace(shape, q.device, dtype)
         elif not workspace.is_cuda or workspace.device != q.device:
             raise ValueError("workspace must be on the same CUDA device as q")
         s = shape.c()

@@ -499,10 +499,11 @@ namespace {
 
 struct BwdWsLayout {
   size_t sorted_off, unsorted_off, delta_off, dq_off, total;
+  size_t deq_off[4];   // MXFP8: exact dequantised q, k, v, dout (bf16 [T, H, d])
   int64_t max_entries;
 };
 
-BwdWsLayout bwd_ws_layout(const attn_shape_t& s) {
+BwdWsLayout bwd_ws_layout(const attn_shape_t& s, attn_dtype_t dtype) {
   BwdWsLayout w{};
   w.max_entries = max_work_entries(s.total_tokens, s.num_seqs);
   w.sorted_off = kWsListOffset;
@@ -511,6 +512,12 @@ BwdWsLayout bwd_ws_layout(const attn_shape_t& s) {
   const size_t rows = static_cast<size_t>(s.total_tokens) * s.num_heads;
   w.dq_off = align_up(w.delta_off + 4 * rows, kWsAlign);
   w.total = align_up(w.dq_off + 4 * rows * s.head_dim, kWsAlign);
+  if (dtype == ATTN_MXFP8) {
+    for (int i = 0; i < 4; ++i) {
+      w.deq_off[i] = w.total;
+      w.total = align_up(w.total + 2 * rows * s.head_dim, kWsAlign);
+    }
+  }
   return w;
 }
 
@@ -549,9 +556,10 @@ attn_status_t bwd_kernel_attributes(int dev) {
 
 extern "C" {
 
-size_t attn_bwd_workspace_size(const attn_shape_t* shape) {
+size_t attn_bwd_workspace_size(const attn_shape_t* shape, attn_dtype_t dtype) {
   if (check_shape(shape) != ATTN_OK) return 0;
-  return bwd_ws_layout(*shape).total;
+  if (dtype != ATTN_BF16 && dtype != ATTN_MXFP8) return 0;
+  return bwd_ws_layout(*shape, dtype).total;
 }
 
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out,
@@ -561,7 +569,7 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        size_t workspace_bytes) {
   const attn_status_t st = check_shape(shape);
   if (st != ATTN_OK) return st;
-  if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_BF16 && dtype != ATTN_MXFP8) return ATTN_ERR_UNSUPPORTED;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
   const attn_shape_t s = *shape;
@@ -573,7 +581,7 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   const void* ptrs[9] = {q, k, v, out, dout, lse, dq, dk, dv};
   for (const void* p : ptrs)
     if (!aligned16(p)) return ATTN_ERR_ALIGNMENT;
-  const BwdWsLayout wl = bwd_ws_layout(s);
+  const BwdWsLayout wl = bwd_ws_layout(s, dtype);
   if (workspace == nullptr || workspace_bytes < wl.total) return ATTN_ERR_WORKSPACE;
   if (!aligned16(workspace)) return ATTN_ERR_ALIGNMENT;
 
@@ -595,6 +603,31 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
       reinterpret_cast<int4*>(ws + wl.sorted_off), reinterpret_cast<int4*>(ws + wl.unsorted_off),
       static_cast<int>(cap));
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+  // 1b. MXFP8: Q, K, V and dO quantised (E4M3, one E8M0 scale per token,
+  //     head and 32 head-dim elements) and exactly dequantised in one
+  //     launch; every product below reads these values, in whichever
+  //     orientation it needs them, so the forward (which quantises Q, K, V
+  //     the same way) and the backward see one set of operands.
+  if (dtype == ATTN_MXFP8) {
+    const void* src[4] = {q, k, v, dout};
+    QuantJobs jobs;
+    jobs.n_blocks = static_cast<long long>(s.total_tokens) * s.num_heads * (s.head_dim / 32);
+    for (int i = 0; i < 4; ++i) {
+      jobs.t[i].x = static_cast<const uint4*>(src[i]);
+      jobs.t[i].codes = nullptr;
+      jobs.t[i].scales = nullptr;
+      jobs.t[i].deq = reinterpret_cast<uint4*>(ws + wl.deq_off[i]);
+    }
+    const long long qgrid = (jobs.n_blocks + 255) / 256;
+    if (qgrid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    quantize_mxfp8_qkv_kernel<<<dim3(static_cast<unsigned>(qgrid), 4), 256, 0, strm>>>(jobs);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    q = ws + wl.deq_off[0];
+    k = ws + wl.deq_off[1];
+    v = ws + wl.deq_off[2];
+    dout = ws + wl.deq_off[3];
+  }
 
   // 2. D = rowsum(dO * O), dQ accumulator cleared
   const long long rows = static_cast<long long>(s.total_tokens) * s.num_heads;

@@ -119,8 +119,9 @@ quantize_mxfp8_kernel(const uint4* __restrict__ x, uint4* __restrict__ codes,
   quantize_block(x, codes, scales, deq, b);
 }
 
-// Q, K and V of one attention call in one launch (blockIdx.y picks the
-// tensor), each with the outputs its consumer reads.
+// The operands of one attention call in one launch (blockIdx.y picks the
+// tensor: Q, K, V, and dO for the backward), each with the outputs its
+// consumer reads.
 struct QuantJob {
   const uint4* x;
   uint4* codes;
@@ -128,7 +129,7 @@ struct QuantJob {
   uint4* deq;
 };
 struct QuantJobs {
-  QuantJob t[3];
+  QuantJob t[4];
   long long n_blocks;   // per tensor
 };
 

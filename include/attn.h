@@ -213,10 +213,12 @@ attn_status_t attn_get_device_error(const void* workspace, void* stream,
 attn_status_t attn_timing_enable(int32_t enable);
 attn_status_t attn_timing_read(float* attention_ms, float* prepass_ms);
 
-/* Bytes of device workspace attn_bwd needs for this shape (0 for an invalid
- * shape): the error word and work lists as for attn_fwd, then D (fp32
- * [H, T]) and the fp32 dQ accumulator ([T, H, d]). */
-size_t attn_bwd_workspace_size(const attn_shape_t* shape);
+/* Bytes of device workspace attn_bwd needs for this shape and dtype (0 for
+ * an invalid shape or dtype): the error word and work lists as for
+ * attn_fwd, then D (fp32 [H, T]) and the fp32 dQ accumulator ([T, H, d]);
+ * for ATTN_MXFP8 also the exactly dequantised q, k, v and dout (bf16
+ * [T, H, d] each). */
+size_t attn_bwd_workspace_size(const attn_shape_t* shape, attn_dtype_t dtype);
 
 /* Exact attention backward: the gradients of attn_fwd's output with respect
  * to q, k and v, given the upstream gradient dout.  The pages print no
@@ -229,9 +231,19 @@ size_t attn_bwd_workspace_size(const attn_shape_t* shape);
  * q, k, v, out, dout: bf16 [T, H, d] (out and lse as attn_fwd wrote them for
  * the same q, k, v, cu_seqlens, causal and scale); lse: fp32 [H, T];
  * dq, dk, dv: bf16 [T, H, d], written.  Same cu_seqlens, shape and causal
- * rules as attn_fwd; dtype must be ATTN_BF16 (ATTN_ERR_UNSUPPORTED
- * otherwise); head dim 64 or 128.  Launches the schedule-build kernel, a
- * kernel computing D and clearing the accumulator, the backward kernel (one
+ * rules as attn_fwd; head dim 64 or 128.
+ * dtype ATTN_MXFP8 is the backward of attn_fwd's MXFP8 path (FLAMIA,
+ * section "FLAMIA Mimarisi ve Temel Tasarım İlkeleri": forward and
+ * backward numerically consistent, quantised operands reused across matrix
+ * orientations, no scale covering a future token): q, k, v and dout are
+ * quantised per token, head and 32 head-dim elements exactly as the forward
+ * quantises q, k, v, and the gradients are those of the attention on the
+ * exactly dequantised operands (passed straight through the quantiser);
+ * out and lse must come from the MXFP8 forward.  One quantisation of each
+ * operand serves every product and orientation.
+ * Launches the schedule-build kernel, for ATTN_MXFP8 one quantisation
+ * kernel for q, k, v and dout, a kernel computing D and clearing the
+ * accumulator, the backward kernel (one
  * 128-key tile of a document and head per work unit; dK and dV accumulate
  * on chip, dQ through fp32 vector reductions, so dq is not bit-reproducible
  * across calls) and the kernel that scales and rounds dQ.  Device faults

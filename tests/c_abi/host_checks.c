@@ -51,10 +51,14 @@ int main(void) {
   check(attn_workspace_size(&big, ATTN_MXFP8) > attn_workspace_size(&big, ATTN_BF16),
         "MXFP8 workspace holds the quantised operands");
   check(attn_workspace_size(&bad_d, ATTN_BF16) == 0, "unsupported head dim: size 0");
-  check(attn_bwd_workspace_size(&big) >=
+  check(attn_bwd_workspace_size(&big, ATTN_BF16) >=
             (size_t)16384 * 32 * 4 + (size_t)16384 * 32 * 128 * 4,
         "backward workspace holds D and the dQ accumulator");
-  check(attn_bwd_workspace_size(&bad_d) == 0, "backward: unsupported head dim: size 0");
+  check(attn_bwd_workspace_size(&big, ATTN_MXFP8) >=
+            attn_bwd_workspace_size(&big, ATTN_BF16) + (size_t)4 * 2 * 16384 * 32 * 128,
+        "MXFP8 backward workspace holds the dequantised operands");
+  check(attn_bwd_workspace_size(&bad_d, ATTN_BF16) == 0,
+        "backward: unsupported head dim: size 0");
 
   /* forward: rejected before launch */
   check(attn_fwd(p16, p16, p16, NULL, p16, (float*)p16, 1, 0.125f, ATTN_BF16, NULL, NULL, p16,
@@ -75,8 +79,12 @@ int main(void) {
 
   /* backward: rejected before launch */
   check(attn_bwd(p16, p16, p16, p16, p16, (const float*)p16, NULL, p16, p16, p16, 1, 0.125f,
-                 ATTN_MXFP8, NULL, &ok, p16, (size_t)1 << 30) == ATTN_ERR_UNSUPPORTED,
-        "backward: MXFP8 not built");
+                 (attn_dtype_t)7, NULL, &ok, p16, (size_t)1 << 30) == ATTN_ERR_UNSUPPORTED,
+        "backward: unknown dtype");
+  check(attn_bwd(p16, p16, p16, p16, p16, (const float*)p16, NULL, p16, p16, p16, 1, 0.125f,
+                 ATTN_MXFP8, NULL, &ok, p16, attn_bwd_workspace_size(&ok, ATTN_BF16)) ==
+            ATTN_ERR_WORKSPACE,
+        "backward: MXFP8 workspace holds more than the bf16 one");
   check(attn_bwd(p16, p16, p16, p16, NULL, (const float*)p16, NULL, p16, p16, p16, 1, 0.125f,
                  ATTN_BF16, NULL, &ok, p16, (size_t)1 << 30) == ATTN_ERR_INVALID_ARG,
         "backward: NULL dout");

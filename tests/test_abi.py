@@ -119,6 +119,9 @@ def test_bwd_workspace_size(L):
     max_entries = 16384 // 128 + 7 + 1
     # lists, D (fp32 [H, T]) and the fp32 dQ accumulator
     assert n >= 256 + 2 * 16 * max_entries + 4 * 16384 * 32 + 4 * 16384 * 32 * 128
+    # MXFP8: plus the dequantised q, k, v and dout
+    assert A.bwd_workspace_size(s, A.ATTN_MXFP8) >= n + 4 * 2 * 16384 * 32 * 128
+    assert A.bwd_workspace_size(s, 7) == 0
     assert A.bwd_workspace_size(A.Shape(16, 1, 1, 96, 16)) == 0
     assert A.bwd_workspace_size(A.Shape(-1, 1, 1, 64, 16)) == 0
 
@@ -127,7 +130,9 @@ def test_bwd_host_checks_return_before_launch(L):
     ok = A.Shape(256, 1, 2, 64, 256)
     assert _bwd(L, None) == 1
     assert _bwd(L, A.Shape(256, 1, 2, 96, 256)) == 2            # d unsupported
-    assert _bwd(L, ok, dtype=1) == 2                            # MXFP8 backward: not built
+    assert _bwd(L, ok, dtype=7) == 2                            # unknown dtype
+    n_bf16 = A.bwd_workspace_size(ok)
+    assert _bwd(L, ok, dtype=1, ws_bytes=n_bf16) == 4           # MXFP8 needs more
     assert _bwd(L, ok, scale=-1.0) == 1
     assert _bwd(L, ok, causal=3) == 1
     assert _bwd(L, A.Shape(256, 2, 2, 64, 100)) == 1            # dense: T != B*N

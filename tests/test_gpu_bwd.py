@@ -15,7 +15,7 @@ import torch
 
 from exact_tiled_attention_39_b200 import attn as A
 from exact_tiled_attention_39_b200 import workloads
-from oracle.attention_bwd import ref_attention_bwd
+from oracle.attention_bwd import ref_attention_bwd, ref_attention_bwd_mxfp8
 
 BWD_REL_MAX = 2e-2
 BWD_REL_MEAN = 2e-3
@@ -30,7 +30,7 @@ def _inputs(lengths, H, d, seed):
     return q, k, v, do
 
 
-def _run(q, k, v, do, cu, causal, scale, max_seqlen, num_seqs=None):
+def _run(q, k, v, do, cu, causal, scale, max_seqlen, num_seqs=None, dtype=A.ATTN_BF16):
     dev = torch.device("cuda:0")
     qd, kd, vd, dod = (t.to(dev).contiguous() for t in (q, k, v, do))
     T, H, d = q.shape
@@ -38,10 +38,10 @@ def _run(q, k, v, do, cu, causal, scale, max_seqlen, num_seqs=None):
     lse = torch.empty((H, T), dtype=torch.float32, device=dev)
     cud = cu.to(dev) if cu is not None else None
     A.attn_fwd(qd, kd, vd, cud, out, lse, causal, scale, max_seqlen=max_seqlen,
-               num_seqs=num_seqs)
+               num_seqs=num_seqs, dtype=dtype)
     dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
     ws = A.attn_bwd(qd, kd, vd, out, dod, lse, cud, dq, dk, dv, causal, scale,
-                    max_seqlen=max_seqlen, num_seqs=num_seqs)
+                    max_seqlen=max_seqlen, num_seqs=num_seqs, dtype=dtype)
     assert A.attn_get_device_error(ws) == 0
     return dq.cpu(), dk.cpu(), dv.cpu()
 
@@ -102,3 +102,67 @@ def test_bwd_bad_seqlens_leaves_outputs():
     assert A.attn_get_device_error(ws) == 5
     for t in (dq, dk, dv):
         assert bool((t == 7.0).all())
+
+
+# ---------------------------------------------------------------- MXFP8
+def _outlier_inputs(lengths, H, d, seed):
+    """Q, K with two outlier channels x20 (the long-context recipe), V and dO
+    plain, all rounded to bf16."""
+    g = torch.Generator().manual_seed(seed)
+    T = sum(lengths)
+    x = [torch.randn((T, H, d), generator=g) for _ in range(4)]
+    for t in x[:2]:
+        t[:, :, 5] *= 20
+        t[:, :, 70 % d] *= 20
+    return [t.to(torch.bfloat16) for t in x]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [True, False])
+def test_bwd_mxfp8_packed_ragged(d, causal):
+    """The MXFP8 backward (out and lse from the MXFP8 forward) against the
+    fp64 gradient oracle of the MXFP8 path (gradients on the exactly
+    dequantised Q, K, V, dO), every element, ragged pack with outliers."""
+    lengths = [1, 130, 0, 300, 129, 64, 256, 44]
+    q, k, v, do = _outlier_inputs(lengths, 2, d, seed=51 + d)
+    scale = 1.0 / math.sqrt(d)
+    cu = workloads.cu_from_lengths(lengths)
+    got = _run(q, k, v, do, cu, causal, scale, max(lengths), dtype=A.ATTN_MXFP8)
+    ref = ref_attention_bwd_mxfp8(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                  do.double().numpy(), cu.numpy(), causal, scale)
+    for gt, rf, n in zip(got, ref, ("dq", "dk", "dv")):
+        _check(gt, rf, n)
+
+
+def test_bwd_mxfp8_long_document():
+    """One 2048-token document with outlier channels, d 128, MXFP8."""
+    q, k, v, do = _outlier_inputs([2048], 2, 128, seed=53)
+    cu = workloads.cu_from_lengths([2048])
+    scale = 1.0 / math.sqrt(128)
+    got = _run(q, k, v, do, cu, True, scale, 2048, dtype=A.ATTN_MXFP8)
+    ref = ref_attention_bwd_mxfp8(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                  do.double().numpy(), cu.numpy(), True, scale)
+    for gt, rf, n in zip(got, ref, ("dq", "dk", "dv")):
+        _check(gt, rf, n)
+
+
+def test_bwd_mxfp8_no_leak_across_documents():
+    """Scales cover one token of one head, so the quantised operands of a
+    document do not depend on any other document: changing every other
+    document's Q, K, V and dO (by large values, which would move any scale
+    shared with them) leaves this document's dK and dV bit-identical and its
+    dQ equal up to the order of the fp32 accumulator's additions."""
+    lengths = [200, 450, 90]
+    q, k, v, do = _outlier_inputs(lengths, 2, 128, seed=55)
+    cu = workloads.cu_from_lengths(lengths)
+    got = _run(q, k, v, do, cu, True, 0.088, 450, dtype=A.ATTN_MXFP8)
+    g = torch.Generator().manual_seed(56)
+    x2 = [t.clone() for t in (q, k, v, do)]
+    for t in x2:
+        t[:200] = (torch.randn(t[:200].shape, generator=g) * 50).bfloat16()
+        t[650:] = (torch.randn(t[650:].shape, generator=g) * 50).bfloat16()
+    got2 = _run(*x2, cu, True, 0.088, 450, dtype=A.ATTN_MXFP8)
+    doc = slice(200, 650)
+    assert torch.equal(got2[1][doc], got[1][doc]) and torch.equal(got2[2][doc], got[2][doc])
+    dq_a, dq_b = got[0][doc].float(), got2[0][doc].float()
+    assert float((dq_a - dq_b).abs().max()) <= 2 ** -7 * float(dq_a.abs().max())
