@@ -1,7 +1,8 @@
 """Benchmark of the exact tiled attention forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload dense_causal|packed_causal|long_outlier|mxfp8_packed|mxfp8_incoherent]
+                    [--workload dense_causal|packed_causal|long_outlier|mxfp8_packed|
+                     mxfp8_incoherent|nvfp4_packed]
                     [--pass fwd|bwd]
 
 One step = one ``attn_fwd`` call through the C ABI (the schedule-build
@@ -254,13 +255,14 @@ class ClockSampler:
 
 KERNEL_TIMING_LAUNCHES = 50       # per-kernel time: median of at least this many launches
 KERNEL_TIMING_MIN_S = 0.05        # ... and of at least this much device time
-EXTRA_WORKLOADS = ("packed_causal", "long_outlier", "mxfp8_packed", "mxfp8_incoherent")
+EXTRA_WORKLOADS = ("packed_causal", "long_outlier", "mxfp8_packed", "mxfp8_incoherent",
+                   "nvfp4_packed")
 
 
 def kernel_name_for(dtype_name: str) -> str:
-    """bf16 runs the two-query-tile kernel, MXFP8 (head dim 128) the
-    block-scaled one."""
-    return "attn_fwd_kernel" if dtype_name == "mxfp8" else "attn_fwd_pair_kernel"
+    """bf16 runs the two-query-tile kernel, MXFP8 and NVFP4 (head dim 128)
+    the block-scaled one."""
+    return "attn_fwd_kernel" if dtype_name in ("mxfp8", "nvfp4") else "attn_fwd_pair_kernel"
 
 
 def measure_workload(A, name, steps, warmup, dev, stream, pg, clk):
@@ -274,7 +276,7 @@ def measure_workload(A, name, steps, warmup, dev, stream, pg, clk):
     inp = workloads.make_inputs(w)
     T, H, d = inp["q"].shape
     causal = True
-    dtype = A.ATTN_MXFP8 if w.dtype == "mxfp8" else A.ATTN_BF16
+    dtype = {"mxfp8": A.ATTN_MXFP8, "nvfp4": A.ATTN_NVFP4}.get(w.dtype, A.ATTN_BF16)
     lengths = inp["lengths"]
     max_seqlen = max(lengths)
     flops = workloads.flops(lengths, H, d, causal)
@@ -331,28 +333,38 @@ def measure_workload(A, name, steps, warmup, dev, stream, pg, clk):
         "ms_step": ms_step, "kernel_ms": statistics.median(per),
         "prepass_ms": statistics.median(pre), "launches_timed": len(per), "err": err,
         "tensors": (q, k, v, cu, out, lse), "step": step,
-        "launches_per_step": 3 if dtype == A.ATTN_MXFP8 else 2,
+        "launches_per_step": 2 if dtype == A.ATTN_BF16 else 3,
     }
+
+
+# Nominal dense tensor rate of each operand type relative to bf16.
+LOWP_RATIO = {"mxfp8": 2.0, "nvfp4": 4.0}
 
 
 def roofline_for(m, peaks, peak_src):
     """Roofline of the attention kernel: algorithmic FLOPs / its median
-    launch time against the measured dense peak of its dtype (fp8 = 2 x the
-    bf16 figure, the nominal ratio)."""
+    launch time against the measured dense bf16 peak.  The block-scaled
+    kernels run Q K^T on low-precision operands (2 x bf16 for E4M3, 4 x for
+    E2M1, the nominal ratios) and P V in bf16, half of the FLOPs each, so
+    their peak is the time-weighted mix 2 / (1 / r + 1); the fraction of the
+    plain low-precision peak (r x bf16) is given as well."""
     peak_key = "bf16_tflops_sustained" if m["ms_total"] * 1e-3 > 1.0 else "bf16_tflops"
-    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
-    fp8 = m["w"].dtype == "mxfp8"
-    if fp8:
-        peak *= 2.0
+    bf16 = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    r = LOWP_RATIO.get(m["w"].dtype)
+    peak = bf16 if r is None else bf16 * 2.0 / (1.0 / r + 1.0)
     achieved = m["flops"] / (m["kernel_ms"] * 1e-3) / 1e12
     kernel = kernel_name_for(m["w"].dtype)
-    return {
+    src = peak_source_name(peak_key, 0)
+    if r is not None:
+        src += (f"; Q K^T at {r:g} x bf16 ({m['w'].dtype} operands), P V at bf16, half the "
+                f"FLOPs each: {2.0 / (1.0 / r + 1.0):.3f} x bf16")
+    out = {
         "bound": "tensor",
         "achieved": round(achieved, 2),
-        "peak": peak,
+        "peak": round(peak, 1),
         "unit": "TFLOP/s",
         "frac": round(achieved / peak, 4),
-        "peak_source": f"{peak_source_name(peak_key, 1 if fp8 else 0)} ({peak_src})",
+        "peak_source": f"{src} ({peak_src})",
         "timed_unit": (f"attention kernel alone (CUDA events around its launch), median of "
                        f"{m['launches_timed']} launches"),
         "kernel_ms": round(m["kernel_ms"], 4),
@@ -361,6 +373,9 @@ def roofline_for(m, peaks, peak_src):
         "traffic": recorded_traffic(m["w"].name, kernel),
         "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
     }
+    if r is not None:
+        out[f"frac_of_{m['w'].dtype}_peak"] = round(achieved / (bf16 * r), 4)
+    return out
 
 
 def bench_ours(args):
@@ -457,7 +472,7 @@ def bench_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "mxfp8" if dtype == A.ATTN_MXFP8 else "bf16",
+        "dtype": w.dtype,
         "data": "synthetic (seeded N(0,1) bf16, see workloads.py)",
         "config": workload_config(w, inp, world),
         "roofline": roof,
@@ -468,7 +483,7 @@ def bench_ours(args):
             "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
         },
-        "gpu_launches": args.steps * (3 if dtype == A.ATTN_MXFP8 else 2),
+        "gpu_launches": args.steps * (2 if dtype == A.ATTN_BF16 else 3),
         "clocks": clk.summary(),
         "device_error": err,
     }
@@ -504,6 +519,7 @@ def cpu_baseline(w, inp, budget_s=15.0):
     from oracle.attention import ref_attention
     from oracle.incoherent import incoherent_operands
     from oracle.mxfp8 import quantize_mxfp8_ref, dequantize_mxfp8_ref
+    from oracle.nvfp4 import dequantize_nvfp4_ref, quantize_nvfp4_ref
 
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
@@ -520,7 +536,10 @@ def cpu_baseline(w, inp, budget_s=15.0):
         k = inp["k"][a:b, h:h + 1].double().numpy()
         v = inp["v"][a:b, h:h + 1].double().numpy()
         scale = inp["scale"]
-        if w.incoherent:
+        if w.dtype == "nvfp4":
+            q, k = (dequantize_nvfp4_ref(*quantize_nvfp4_ref(x)) for x in (q, k))
+            v = dequantize_mxfp8_ref(*quantize_mxfp8_ref(v))
+        elif w.incoherent:
             q, k, v, scale = incoherent_operands(q, k, v, scale, inp["signs"].numpy())
         elif w.dtype == "mxfp8":
             q, k, v = (dequantize_mxfp8_ref(*quantize_mxfp8_ref(x)) for x in (q, k, v))
@@ -575,8 +594,8 @@ def bench_ours_bwd(args):
     pg = init_group("nccl", dev)
 
     w = workloads.get(args.workload)
-    if w.incoherent:
-        raise SystemExit("--pass bwd: the backward has no incoherent-processing form")
+    if w.incoherent or w.dtype == "nvfp4":
+        raise SystemExit("--pass bwd: the backward covers the bf16 and MXFP8 paths")
     dtype = A.ATTN_MXFP8 if w.dtype == "mxfp8" else A.ATTN_BF16
     inp = workloads.make_inputs(w)
     T, H, d = inp["q"].shape

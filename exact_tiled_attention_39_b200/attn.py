@@ -12,16 +12,17 @@ from dataclasses import dataclass
 
 import torch
 
-__all__ = ["ATTN_BF16", "ATTN_MXFP8", "AttnError", "lib", "workspace_size", "attn_fwd",
+__all__ = ["ATTN_BF16", "ATTN_MXFP8", "ATTN_NVFP4", "AttnError", "lib", "workspace_size", "attn_fwd",
            "attn_fwd_noalloc", "attn_quantize_mxfp8", "attn_get_device_error", "status_string",
            "make_workspace", "attn_timing_enable", "attn_timing_read", "bwd_workspace_size",
            "make_bwd_workspace", "attn_bwd", "attn_quantize_mxfp8_rotated",
-           "attn_fwd_incoherent", "LIB_PATH", "EXPORTED_SYMBOLS"]
+           "attn_fwd_incoherent", "attn_quantize_nvfp4", "LIB_PATH", "EXPORTED_SYMBOLS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 
 ATTN_BF16 = 0
 ATTN_MXFP8 = 1
+ATTN_NVFP4 = 2
 
 STATUS = {
     0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_ALIGNMENT",
@@ -32,7 +33,7 @@ EXPORTED_SYMBOLS = ("attn_workspace_size", "attn_fwd", "attn_quantize_mxfp8",
                     "attn_get_device_error", "attn_status_string", "attn_abi_version",
                     "attn_fwd_noalloc", "attn_timing_enable", "attn_timing_read",
                     "attn_bwd_workspace_size", "attn_bwd", "attn_quantize_mxfp8_rotated",
-                    "attn_fwd_incoherent")
+                    "attn_fwd_incoherent", "attn_quantize_nvfp4")
 
 
 class AttnError(RuntimeError):
@@ -86,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_incoherent.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_float,
                                           vp, vp, ctypes.POINTER(_Shape), vp, sz]
         L.attn_fwd_incoherent.restype = ctypes.c_int
+        L.attn_quantize_nvfp4.argtypes = [vp, vp, vp, i64, i32, vp]
+        L.attn_quantize_nvfp4.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -270,6 +273,19 @@ def attn_quantize_mxfp8(x, codes, scales, stream=None):
                                    _stream_handle(stream, x.device))
     if rc != 0:
         raise AttnError(rc, "attn_quantize_mxfp8")
+
+
+def attn_quantize_nvfp4(x, codes, scales, stream=None):
+    """NVFP4 quantisation of a bf16 [rows, cols] CUDA tensor (any leading
+    shape; cols a multiple of 16): codes uint8 [rows, cols / 2] (two E2M1
+    codes per byte, low nibble first), scales uint8 [rows, cols / 16]
+    (unsigned E4M3)."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    rc = lib().attn_quantize_nvfp4(_ptr(x), _ptr(codes), _ptr(scales), rows, cols,
+                                   _stream_handle(stream, x.device))
+    if rc != 0:
+        raise AttnError(rc, "attn_quantize_nvfp4")
 
 
 def attn_quantize_mxfp8_rotated(x, signs, codes, scales, stream=None):

@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "incoherent.cuh"
 #include "quant_mxfp8.cuh"
+#include "quant_nvfp4.cuh"
 #include "schedule.cuh"
 
 namespace attn {
@@ -84,10 +85,14 @@ int64_t sort_capacity_for(int64_t max_entries) {
 
 struct WsLayout {
   size_t sorted_off, unsorted_off, mx_off, total;
-  // MXFP8: per operand (q, k, v) E4M3 codes, E8M0 scales, bf16 dequantised copy
+  // MXFP8 / NVFP4: per operand (q, k, v) codes, scales, bf16 dequantised copy
   size_t codes_off[3], scales_off[3], deq_off[3];
   int64_t max_entries;
 };
+
+bool valid_fwd_dtype(attn_dtype_t dtype) {
+  return dtype == ATTN_BF16 || dtype == ATTN_MXFP8 || dtype == ATTN_NVFP4;
+}
 
 WsLayout ws_layout(const attn_shape_t& s, attn_dtype_t dtype) {
   WsLayout w{};
@@ -96,13 +101,16 @@ WsLayout ws_layout(const attn_shape_t& s, attn_dtype_t dtype) {
   w.unsorted_off = align_up(w.sorted_off + 16 * static_cast<size_t>(w.max_entries), kWsAlign);
   w.mx_off = align_up(w.unsorted_off + 16 * static_cast<size_t>(w.max_entries), kWsAlign);
   w.total = w.mx_off;
-  if (dtype == ATTN_MXFP8) {
+  if (dtype == ATTN_MXFP8 || dtype == ATTN_NVFP4) {
     const size_t elems = static_cast<size_t>(s.total_tokens) * s.num_heads * s.head_dim;
+    // MXFP8: one E4M3 byte per element, one E8M0 scale per 32; NVFP4 (q and
+    // k): half a byte per element, one UE4M3 scale per 16
+    const bool nv = dtype == ATTN_NVFP4;
     for (int i = 0; i < 3; ++i) {
       w.codes_off[i] = w.total;
-      w.total = align_up(w.total + elems, kWsAlign);
+      w.total = align_up(w.total + (nv ? elems / 2 : elems), kWsAlign);
       w.scales_off[i] = w.total;
-      w.total = align_up(w.total + elems / 32, kWsAlign);
+      w.total = align_up(w.total + (nv ? elems / 16 : elems / 32), kWsAlign);
       w.deq_off[i] = w.total;
       w.total = align_up(w.total + 2 * elems, kWsAlign);
     }
@@ -138,9 +146,12 @@ attn_status_t device_info(int* dev_out, DeviceInfo* info) {
   if (!d.ready) {
     if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<128, true>,
+    if (cudaFuncSetAttribute(attn_fwd_kernel<128, kQkMx8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FwdLayout<128, true>::kBytes) != cudaSuccess ||
+                             FwdLayout<128, kQkMx8>::kBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel<128, kQkNv4>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FwdLayout<128, kQkNv4>::kBytes) != cudaSuccess ||
         cudaFuncSetAttribute(attn_fwd_pair_kernel<64>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              PairLayout<64>::kBytes) != cudaSuccess ||
@@ -175,6 +186,21 @@ bool encode_qkv_map(CUtensorMap* m, const void* base, int T, int H, int d, int e
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over packed E2M1 codes [T, H, d / 2 bytes]: box = the d / 2 bytes
+// of a row (64 for d = 128) x 1 head x 128 tokens, 64-byte swizzle.
+bool encode_fp4_map(CUtensorMap* m, const void* base, int T, int H, int d) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d / 2), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d / 2),
+                                 static_cast<cuuint64_t>(H) * (d / 2)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(d / 2), 1, static_cast<cuuint32_t>(kBlockM)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 }  // namespace attn
 
@@ -200,7 +226,7 @@ const char* attn_status_string(attn_status_t s) {
 
 size_t attn_workspace_size(const attn_shape_t* shape, attn_dtype_t dtype) {
   if (check_shape(shape) != ATTN_OK) return 0;
-  if (dtype != ATTN_BF16 && dtype != ATTN_MXFP8) return 0;
+  if (!valid_fwd_dtype(dtype)) return 0;
   return ws_layout(*shape, dtype).total;
 }
 
@@ -234,7 +260,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
                        void* workspace, size_t workspace_bytes) {
   const attn_status_t st = check_shape(shape);
   if (st != ATTN_OK) return st;
-  if (dtype != ATTN_BF16 && dtype != ATTN_MXFP8) return ATTN_ERR_UNSUPPORTED;
+  if (!valid_fwd_dtype(dtype)) return ATTN_ERR_UNSUPPORTED;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
   const attn_shape_t s = *shape;
@@ -258,7 +284,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
 
   // The block-scaled kernel (MXFP8, d = 128) takes one query tile per unit;
   // the bf16 kernel two.
-  const bool fp8_kernel = dtype == ATTN_MXFP8 && s.head_dim == 128;
+  const bool nv4 = dtype == ATTN_NVFP4;
+  const bool fp8_kernel = (dtype == ATTN_MXFP8 || nv4) && s.head_dim == 128;
   const bool pair_kernel = !fp8_kernel;
   timing_mark(0, strm);
   // 1. schedule (validates cu_seqlens, writes the work list and its length)
@@ -303,6 +330,27 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
     v = ws + wl.deq_off[2];
     // (Q M)(K M)^T = d Q K^T: exact division by the power of two d
     scale /= static_cast<float>(s.head_dim);
+  } else if (nv4) {
+    // Mixed NVFP4 / FP8 path: Q and K to NVFP4 (packed E2M1 codes and UE4M3
+    // scales for the block-scaled kernel; the exact dequantised values for
+    // head dim 64), V to MXFP8 (exact dequantised bf16), one launch.
+    MixedQuantJobs jobs;
+    const void* src[3] = {q, k, v};
+    for (int i = 0; i < 3; ++i) {
+      jobs.x[i] = static_cast<const uint4*>(src[i]);
+      jobs.deq[i] = (i == 2 || !fp8_kernel) ? reinterpret_cast<uint4*>(ws + wl.deq_off[i]) : nullptr;
+    }
+    for (int i = 0; i < 2; ++i) {
+      jobs.codes[i] = fp8_kernel ? reinterpret_cast<uint2*>(ws + wl.codes_off[i]) : nullptr;
+      jobs.scales[i] = fp8_kernel ? ws + wl.scales_off[i] : nullptr;
+    }
+    jobs.n16 = static_cast<long long>(s.total_tokens) * s.num_heads * (s.head_dim / 16);
+    const long long qgrid = (jobs.n16 + 255) / 256;
+    if (qgrid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    quantize_nvfp4_qk_mxfp8_v_kernel<<<dim3(static_cast<unsigned>(qgrid), 3), 256, 0, strm>>>(jobs);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    for (int i = 0; i < 2; ++i) qk_src[i] = ws + (fp8_kernel ? wl.codes_off[i] : wl.deq_off[i]);
+    v = ws + wl.deq_off[2];
   } else if (dtype == ATTN_MXFP8) {
     // One launch for all three tensors.  The block-scaled kernel reads the
     // codes and scales of Q and K and the exact dequantised V; the head-dim
@@ -330,10 +378,15 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
   // 3. attention
   const int qk_elem = fp8_kernel ? 1 : 2;
   CUtensorMap tq, tk, tv;
-  if (!encode_qkv_map(&tq, qk_src[0], s.total_tokens, s.num_heads, s.head_dim, qk_elem) ||
-      !encode_qkv_map(&tk, qk_src[1], s.total_tokens, s.num_heads, s.head_dim, qk_elem) ||
-      !encode_qkv_map(&tv, v, s.total_tokens, s.num_heads, s.head_dim, 2))
+  if (fp8_kernel && nv4) {
+    if (!encode_fp4_map(&tq, qk_src[0], s.total_tokens, s.num_heads, s.head_dim) ||
+        !encode_fp4_map(&tk, qk_src[1], s.total_tokens, s.num_heads, s.head_dim))
+      return ATTN_ERR_CUDA;
+  } else if (!encode_qkv_map(&tq, qk_src[0], s.total_tokens, s.num_heads, s.head_dim, qk_elem) ||
+             !encode_qkv_map(&tk, qk_src[1], s.total_tokens, s.num_heads, s.head_dim, qk_elem)) {
     return ATTN_ERR_CUDA;
+  }
+  if (!encode_qkv_map(&tv, v, s.total_tokens, s.num_heads, s.head_dim, 2)) return ATTN_ERR_CUDA;
   FwdParams fp;
   fp.out = out;
   fp.lse = lse;
@@ -364,9 +417,12 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
   cfg.numAttrs = 1;
   cudaError_t e;
   timing_mark(1, strm);
-  if (fp8_kernel) {
-    cfg.dynamicSmemBytes = FwdLayout<128, true>::kBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, true>, tq, tk, tv, fp);
+  if (fp8_kernel && nv4) {
+    cfg.dynamicSmemBytes = FwdLayout<128, kQkNv4>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, kQkNv4>, tq, tk, tv, fp);
+  } else if (fp8_kernel) {
+    cfg.dynamicSmemBytes = FwdLayout<128, kQkMx8>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, kQkMx8>, tq, tk, tv, fp);
   } else if (s.head_dim == 128) {
     cfg.dynamicSmemBytes = PairLayout<128>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<128>, tq, tk, tv, fp);
@@ -718,5 +774,24 @@ extern "C" attn_status_t attn_quantize_mxfp8_rotated(const void* x, const float*
   else
     quantize_mxfp8_rotated_kernel<64><<<static_cast<unsigned>(grid), 128, 0, strm>>>(
         static_cast<const uint4*>(x), signs, reinterpret_cast<uint4*>(codes), scales, rows);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ===========================================================================
+// NVFP4 quantisation pre-pass on its own: attn_quantize_nvfp4.
+// ===========================================================================
+
+extern "C" attn_status_t attn_quantize_nvfp4(const void* x, uint8_t* codes, uint8_t* scales,
+                                             int64_t rows, int32_t cols, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 16 != 0) return ATTN_ERR_INVALID_ARG;
+  if (rows == 0) return ATTN_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(codes) & 7u) != 0) return ATTN_ERR_ALIGNMENT;
+  const long long n_blocks = rows * static_cast<long long>(cols / 16);
+  const long long grid = (n_blocks + 255) / 256;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  quantize_nvfp4_kernel<<<static_cast<unsigned>(grid), 256, 0,
+                          static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(x), reinterpret_cast<uint2*>(codes), scales, nullptr, n_blocks);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -67,8 +67,8 @@ struct FwdParams {
   const int32_t* ws_header;  // error word, work-list length, unit counter
   const int4* work;          // work list
   int32_t* err;              // error word (device)
-  const uint32_t* q_scales;  // MXFP8: E8M0 words [T, H] (4 scales per word)
-  const uint32_t* k_scales;
+  const uint32_t* q_scales;  // MXFP8: E8M0 words [T, H] (4 scales per word);
+  const uint32_t* k_scales;  // NVFP4: UE4M3 words [T, H, 2] (4 scales per word)
   int total_tokens;
   int num_heads;
   int head_groups;           // unit order: heads in this many groups (see common.cuh)
@@ -110,17 +110,30 @@ constexpr float kExp2C1 = 6.951168180e-01f;
 constexpr float kExp2C2 = 2.276448607e-01f;
 constexpr float kExp2C3 = 7.706713676e-02f;
 
-template <int D, bool kFp8>
+// Operand format of the score product Q K^T: bf16, MXFP8 (E4M3 codes, one
+// E8M0 scale per 32 elements) or NVFP4 (E2M1 codes two per byte, one
+// unsigned E4M3 scale per 16 elements).
+constexpr int kQkBf16 = 0, kQkMx8 = 1, kQkNv4 = 2;
+
+template <int D, int kQk>
 struct FwdLayout {
+  static constexpr bool kFp8 = kQk != kQkBf16;                // Q, K as block-scaled codes
+  static constexpr bool kNv4 = kQk == kQkNv4;
   static_assert(D == 64 || D == 128, "head dim 64 or 128");
-  static_assert(!kFp8 || D == 128, "the MXFP8 kernel is built for head dim 128");
-  static constexpr int kQKChunks = kFp8 ? 1 : D / 64;        // 128-byte chunks per Q/K row
+  static_assert(!kFp8 || D == 128, "the block-scaled kernel is built for head dim 128");
+  static constexpr int kQKChunks = kFp8 ? 1 : D / 64;         // swizzle-wide chunks per Q/K row
+  static constexpr int kQKRowBytes = kNv4 ? 64 : 128;         // bytes of a row in one chunk
   static constexpr int kVChunks = D / 64;                     // V is bf16
   static constexpr int kChunkBytes = kBlockM * 128;           // 128 rows x 128 bytes
-  static constexpr int kQBytes = kQKChunks * kChunkBytes;
-  static constexpr int kKBytes = kQKChunks * kChunkBytes;
+  static constexpr int kQKChunkBytes = kBlockM * kQKRowBytes;
+  static constexpr int kQBytes = kQKChunks * kQKChunkBytes;
+  static constexpr int kKBytes = kQKChunks * kQKChunkBytes;
   static constexpr int kVBytes = kVChunks * kChunkBytes;
-  static constexpr int kSfBytes = 512;                        // 128 rows x 4 scale bytes
+  // Scale blocks of a tile: 32 rows x 16 bytes each, one per 32-bit scale
+  // word of a row (MXFP8: 4 E8M0 bytes cover the 128 elements; NVFP4: two
+  // words of 4 UE4M3 bytes, one per 64 elements).
+  static constexpr int kSfWords = kNv4 ? 2 : 1;
+  static constexpr int kSfBytes = 512 * kSfWords;
   static constexpr int kSlotBytes = kVBytes;                  // a V tile, or a K tile + scales
   static_assert(kKBytes + (kFp8 ? kSfBytes : 0) <= kSlotBytes, "K tile must fit a slot");
   static constexpr int kQOff = 0;
@@ -157,7 +170,8 @@ struct FwdLayout {
   static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
   static_assert(kBytes - kStatsOff <= kReserve, "reserve too small");
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kTmemO = 256, kTmemSfa = 384, kTmemSfb = 388;
+  static constexpr uint32_t kTmemO = 256, kTmemSfa = 384;
+  static constexpr uint32_t kTmemSfb = kTmemSfa + 4 * kSfWords;   // + 4 * kSfWords * buffer
 };
 
 // Bounded waits.  A wait gives up when the CTA's abort flag is raised or
@@ -265,6 +279,28 @@ __host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t sf_id) {
          | (sf_id << 29);                     // A scale id
 }
 
+// Instruction descriptor for the block-scaled E2M1 x E2M1 product (fp32
+// accumulate, unsigned E4M3 scales, one per 16 elements, M = N = 128,
+// K = 64): the scale ids are 0, each instruction reads a whole 32-bit scale
+// word per row.
+__host__ __device__ constexpr uint32_t idesc_nvf4() {
+  return (1u << 7) | (1u << 10)               // A, B format: E2M1
+         | (static_cast<uint32_t>(kBlockN >> 3) << 17)
+         | (0u << 23)                         // scale format: UE4M3
+         | (static_cast<uint32_t>(kBlockM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_nvf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t sfa, uint32_t sfb,
                                             uint32_t accumulate) {
@@ -287,11 +323,13 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-template <int D, bool kFp8>
+template <int D, int kQk>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Lay = FwdLayout<D, kFp8>;
+  using Lay = FwdLayout<D, kQk>;
+  constexpr bool kFp8 = Lay::kFp8;
+  constexpr bool kNv4 = Lay::kNv4;
   // The kernel has no static shared memory, so the dynamic block starts at
   // the CTA's (1024-byte aligned) shared window; the 128-byte swizzle needs
   // that alignment.  Checked anyway: a misaligned base records an error and
@@ -584,16 +622,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t slot = sbase + Lay::kRingOff + s * Lay::kSlotBytes;
         const int row0 = ui.doc_start + kBlockN * j;
         if (kFp8 && kind == 0) {
-          // Scale block of the K tile: lane m0 writes keys m0 + 32 c, c = 0..3,
-          // as 16 bytes at offset 16 m0 (the layout tcgen05.cp replicates).
-          uint32_t wv[4];
+          // Scale blocks of the K tile, one per scale word w of a row: lane
+          // m0 writes keys m0 + 32 c, c = 0..3, as 16 bytes at offset
+          // 512 w + 16 m0 (the layout tcgen05.cp replicates).
 #pragma unroll
-          for (int cq = 0; cq < 4; ++cq) {
-            const int tok = row0 + lane + 32 * cq;
-            wv[cq] = tok < p.total_tokens ? p.k_scales[static_cast<long long>(tok) * H + ui.head] : 0u;
+          for (int w = 0; w < Lay::kSfWords; ++w) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int cq = 0; cq < 4; ++cq) {
+              const int tok = row0 + lane + 32 * cq;
+              wv[cq] = tok < p.total_tokens
+                           ? p.k_scales[(static_cast<long long>(tok) * H + ui.head) * Lay::kSfWords + w]
+                           : 0u;
+            }
+            *reinterpret_cast<uint4*>(smem + Lay::kRingOff + s * Lay::kSlotBytes + Lay::kKBytes +
+                                      512 * w + 16 * lane) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
           }
-          *reinterpret_cast<uint4*>(smem + Lay::kRingOff + s * Lay::kSlotBytes + Lay::kKBytes +
-                                    16 * lane) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
           fence_proxy_async_smem();
           __syncwarp();
         }
@@ -602,10 +646,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const int bytes = kind == 0 ? Lay::kKBytes : Lay::kVBytes;
           ptx::mbar_arrive_expect_tx(bar(Lay::kKVFull + s), bytes);
           for (int cq = 0; cq < chunks; ++cq)
-            ptx::tma_load_3d(slot + cq * Lay::kChunkBytes,
+            ptx::tma_load_3d(slot + cq * (kind == 0 ? Lay::kQKChunkBytes : Lay::kChunkBytes),
                              kind == 0 ? static_cast<const void*>(&tm_k)
                                        : static_cast<const void*>(&tm_v),
-                             bar(Lay::kKVFull + s), cq * (kind == 0 && kFp8 ? 128 : 64),
+                             bar(Lay::kKVFull + s), kind == 0 ? cq * Lay::kQKRowBytes / (kFp8 ? 1 : 2) : cq * 64,
                              ui.head, row0);
         }
         __syncwarp();
@@ -657,22 +701,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!(ok = wait_warp(bar(Lay::kQEmpty), (q_it & 1) ^ 1, ctl))) break;
         const int qrow0 = ui.doc_start + kBlockM * ui.qb;
         if constexpr (kFp8) {
-          uint32_t wv[4];
 #pragma unroll
-          for (int cq = 0; cq < 4; ++cq) {
-            const int tok = qrow0 + lane + 32 * cq;
-            wv[cq] = tok < p.total_tokens ? p.q_scales[static_cast<long long>(tok) * H + ui.head] : 0u;
+          for (int w = 0; w < Lay::kSfWords; ++w) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int cq = 0; cq < 4; ++cq) {
+              const int tok = qrow0 + lane + 32 * cq;
+              wv[cq] = tok < p.total_tokens
+                           ? p.q_scales[(static_cast<long long>(tok) * H + ui.head) * Lay::kSfWords + w]
+                           : 0u;
+            }
+            *reinterpret_cast<uint4*>(smem + Lay::kSfaOff + 512 * w + 16 * lane) =
+                make_uint4(wv[0], wv[1], wv[2], wv[3]);
           }
-          *reinterpret_cast<uint4*>(smem + Lay::kSfaOff + 16 * lane) =
-              make_uint4(wv[0], wv[1], wv[2], wv[3]);
           fence_proxy_async_smem();
           __syncwarp();
         }
         if (lane == 0) {
           ptx::mbar_arrive_expect_tx(bar(Lay::kQFull), Lay::kQBytes);
           for (int cq = 0; cq < Lay::kQKChunks; ++cq)
-            ptx::tma_load_3d(sbase + Lay::kQOff + cq * Lay::kChunkBytes, &tm_q, bar(Lay::kQFull),
-                             cq * (kFp8 ? 128 : 64), ui.head, qrow0);
+            ptx::tma_load_3d(sbase + Lay::kQOff + cq * Lay::kQKChunkBytes, &tm_q, bar(Lay::kQFull),
+                             cq * Lay::kQKRowBytes / (kFp8 ? 1 : 2), ui.head, qrow0);
         }
         __syncwarp();
         ++q_it;
@@ -702,6 +751,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       constexpr uint32_t kIdescS = ptx::idesc_bf16(kBlockM, kBlockN, 0);
       constexpr uint32_t kIdescO = ptx::idesc_bf16(kBlockM, D, 1);
       constexpr uint32_t kDescHi = ptx::sdesc_hi_sw128(1024);
+      // NVFP4 Q and K rows are 64 bytes: 64-byte swizzle, 8-row groups 512 B apart
+      constexpr uint32_t kQkDescHi = kNv4 ? ptx::sdesc_hi_sw64(512) : kDescHi;
       const uint32_t q_lo = ptx::sdesc_lo(sbase + Lay::kQOff, 16);
       const uint32_t ring_lo = ptx::sdesc_lo(sbase + Lay::kRingOff, 16);
       const uint32_t v_lbo = static_cast<uint32_t>(Lay::kChunkBytes - 16) >> 4 << 16;
@@ -719,15 +770,34 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!(ok = wait_one(bar(Lay::kQFull), q_ph, ctl))) break;
         q_ph ^= 1;
         ptx::tc_fence_after();
-        if constexpr (kFp8)
-          tmem_cp_32x128b_x4(tmem + Lay::kTmemSfa, sf_copy_desc(sbase + Lay::kSfaOff));
+        if constexpr (kFp8) {
+#pragma unroll
+          for (int w = 0; w < Lay::kSfWords; ++w)
+            tmem_cp_32x128b_x4(tmem + Lay::kTmemSfa + 4 * w,
+                               sf_copy_desc(sbase + Lay::kSfaOff + 512 * w));
+        }
         // S for global step gs from the K tile in ring stage st.  It
         // overwrites P_{gs-2}, so it is issued after P_{gs-2} V_{gs-2} (the
         // tensor pipe keeps issue order).
         auto score = [&](uint32_t gs, uint32_t st) -> bool {
           const uint32_t buf = gs & 1;
           const uint32_t b_lo = ring_lo + st * (Lay::kSlotBytes >> 4);
-          if constexpr (kFp8) {
+          if constexpr (kNv4) {
+            const uint32_t sfb = tmem + Lay::kTmemSfb + 4 * Lay::kSfWords * buf;
+#pragma unroll
+            for (int w = 0; w < Lay::kSfWords; ++w)
+              tmem_cp_32x128b_x4(sfb + 4 * w,
+                                 sf_copy_desc(sbase + Lay::kRingOff + st * Lay::kSlotBytes +
+                                              Lay::kKBytes + 512 * w));
+            // two K = 64 products (32 bytes of packed E2M1 each) per tile
+#pragma unroll
+            for (int kk = 0; kk < D / 64; ++kk) {
+              const uint32_t off = (kk * 32) >> 4;
+              mma_nvf4_ss(tmem + buf * 128, ptx::sdesc_join(q_lo + off, kQkDescHi),
+                          ptx::sdesc_join(b_lo + off, kQkDescHi), idesc_nvf4(),
+                          tmem + Lay::kTmemSfa + 4 * kk, sfb + 4 * kk, kk > 0 ? 1u : 0u);
+            }
+          } else if constexpr (kFp8) {
             const uint32_t sfb = tmem + Lay::kTmemSfb + 4 * buf;
             tmem_cp_32x128b_x4(sfb, sf_copy_desc(sbase + Lay::kRingOff + st * Lay::kSlotBytes +
                                                  Lay::kKBytes));

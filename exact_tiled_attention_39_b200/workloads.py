@@ -71,6 +71,12 @@ WORKLOADS = {
         outlier_channels=(5, 70), outlier_factor=20.0, dtype="mxfp8",
         description="packed as packed_causal (seed 4) with the outlier "
                     "channels of long_outlier, MXFP8"),
+    "nvfp4_packed": Workload(
+        name="nvfp4_packed", seed=4, heads=32, head_dim=128, causal=(True,),
+        pack_tokens=16384, doc_len_range=(128, 4096),
+        outlier_channels=(5, 70), outlier_factor=20.0, dtype="nvfp4",
+        description="the mxfp8_packed inputs on the mixed path: Q, K in NVFP4, "
+                    "V in MXFP8"),
     "mxfp8_incoherent": Workload(
         name="mxfp8_incoherent", seed=4, heads=32, head_dim=128, causal=(True,),
         pack_tokens=16384, doc_len_range=(128, 4096),

@@ -65,11 +65,18 @@ extern "C" {
 
 typedef enum {
   ATTN_BF16 = 0,  /* bf16 operands, bf16 tensor-core products, fp32 softmax   */
-  ATTN_MXFP8 = 1  /* bf16 inputs quantised in-call to E4M3 + E8M0 (per token,
+  ATTN_MXFP8 = 1, /* bf16 inputs quantised in-call to E4M3 + E8M0 (per token,
                      head and 32 head-dim elements).  d = 128: Q K^T is a
                      block-scaled E4M3 product; P V runs in bf16 on the exact
                      dequantisation of V.  d = 64: every product runs in bf16
                      on the exactly dequantised Q, K and V (same values)     */
+  ATTN_NVFP4 = 2  /* the mixed NVFP4 / FP8 path (forward only): bf16 inputs
+                     quantised in-call, Q and K to NVFP4 (E2M1, one unsigned
+                     E4M3 scale per token, head and 16 head-dim elements; see
+                     attn_quantize_nvfp4), V to MXFP8.  d = 128: Q K^T is a
+                     block-scaled E2M1 product; P V runs in bf16 on the
+                     exact dequantisation of V.  d = 64: every product in
+                     bf16 on the exactly dequantised operands             */
 } attn_dtype_t;
 
 typedef enum {
@@ -172,6 +179,20 @@ attn_status_t attn_fwd_noalloc(const void* q, const void* k, const void* v,
  * [0, 254]; an all-zero block gets 127.  Elements: x / 2^(c-127) rounded to
  * nearest E4M3 (ties to even, saturating at 448).  Asynchronous. */
 attn_status_t attn_quantize_mxfp8(const void* x, uint8_t* codes, uint8_t* scales, int64_t rows,
+                                  int32_t cols, void* stream);
+
+/* The NVFP4 quantisation pre-pass of the mixed NVFP4 / FP8 path on its own
+ * (FLAMIA section "FLAMIA Mimarisi ve Temel Tasarım İlkeleri" names the
+ * mixed path beside MXFP8).  x: bf16 [rows, cols] device, 16-byte aligned,
+ * cols a multiple of 16; codes: uint8 [rows, cols / 2], 8-byte aligned, two
+ * E2M1 codes per byte (element 2i in bits 0-3, 2i + 1 in bits 4-7; code =
+ * sign << 3 | magnitude index of 0, 0.5, 1, 1.5, 2, 3, 4, 6); scales: uint8
+ * [rows, cols / 16], unsigned E4M3 (one per 16 elements of a row).  Scale
+ * rule: the smallest positive E4M3 value S with amax <= 6 S (448 past
+ * 6 * 448; 1.0 for a block of zeros); no per-tensor scale.  Elements: the
+ * fp32 quotient x / S (IEEE division) rounded to the nearest E2M1 value,
+ * ties to even, saturating at 6, sign kept.  Asynchronous. */
+attn_status_t attn_quantize_nvfp4(const void* x, uint8_t* codes, uint8_t* scales, int64_t rows,
                                   int32_t cols, void* stream);
 
 /* The MXFP8 pre-pass with incoherent processing ("FlashAttention, pelatihan

@@ -51,6 +51,10 @@ def test_workspace_size(L):
     max_entries = 16384 // 128 + 7 + 1
     assert n_bf16 >= 256 + 2 * 16 * max_entries
     assert n_mx >= n_bf16 + 3 * 16384 * 32 * 128 + 3 * 16384 * 32 * 4
+    n_nv = A.workspace_size(s, A.ATTN_NVFP4)
+    # packed E2M1 codes and UE4M3 scales of q and k, exact bf16 v
+    assert n_nv >= n_bf16 + 2 * (16384 * 32 * 64 + 16384 * 32 * 8) + 2 * 16384 * 32 * 128
+    assert A.workspace_size(s, 3) == 0                              # dtype unsupported
     assert A.workspace_size(A.Shape(16, 1, 1, 96, 16)) == 0       # d unsupported
     assert A.workspace_size(A.Shape(-1, 1, 1, 64, 16)) == 0
 
@@ -170,3 +174,12 @@ def test_incoherent_forward_host_checks(L):
     assert call(None, vp(16)) == 1                # no shape
     assert call(ok, vp(16), ws_bytes=64) == 4     # workspace too small (MXFP8 layout)
     assert call(empty, None) == 0                 # T == 0: no-op
+
+
+def test_nvfp4_quantiser_host_checks(L):
+    vp = ctypes.c_void_p
+    assert L.attn_quantize_nvfp4(None, None, None, 0, 64, None) == 0         # empty
+    assert L.attn_quantize_nvfp4(None, None, None, 4, 40, None) == 1         # cols % 16
+    assert L.attn_quantize_nvfp4(vp(16), vp(16), None, 4, 64, None) == 1     # scales NULL
+    assert L.attn_quantize_nvfp4(vp(24), vp(16), vp(16), 4, 64, None) == 3   # x misaligned
+    assert L.attn_quantize_nvfp4(vp(16), vp(12), vp(16), 4, 64, None) == 3   # codes misaligned
