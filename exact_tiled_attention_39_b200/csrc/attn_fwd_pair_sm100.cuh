@@ -18,15 +18,10 @@
 //
 //   warps 0..3    softmax of tile A (184 registers): one thread per query
 //                 row reads its 128 scores from TMEM, masks, updates m and l,
-//                 and writes P (bf16) over the first 64 columns of its
-//                 scores.  When the row maximum grew by more than 2^8 it
-//                 takes the new maximum and hands the rescale factor of O_A
-//                 to the correction warps (lazy rescale).
-//   warps 4..7    softmax of tile B.  The two tiles' exponential phases take
-//                 turns on each SM sub-partition.
-//   warps 8..11   correction and epilogue (64 registers): rescale O_t when
-//                 the softmax asks for it, off the softmax's path; at the
-//                 end of a tile, O_t / l_round -> bf16 and the lse.
+//                 writes P (bf16) over the first 64 columns of its scores and
+//                 rescales O_A when the row maximum grew by more than 2^8.
+//   warps 4..7    softmax of tile B.
+//   warps 8..11   epilogue (64 registers): O_t / l_round -> bf16, lse.
 //   warp 12       producer (80 registers): claims units, TMA loads of Q_A,
 //                 Q_B and of K_j, V_j into a ring of shared-memory slots.
 //   warp 13       MMA issuer (one thread).
@@ -48,15 +43,6 @@ namespace attn {
 #define ATTN_FAULT_DROP_FIRST_SCORE_COMMIT 0
 #endif
 constexpr bool kFaultDropFirstScoreCommit = ATTN_FAULT_DROP_FIRST_SCORE_COMMIT != 0;
-
-#ifndef ATTN_PINGPONG
-#define ATTN_PINGPONG 0
-#endif
-constexpr bool kPingPong = ATTN_PINGPONG != 0;
-#ifndef ATTN_CORRECTION_WG
-#define ATTN_CORRECTION_WG 1
-#endif
-constexpr bool kCorrectionWG = ATTN_CORRECTION_WG != 0;
 
 constexpr int kPairThreads = 512;
 constexpr uint32_t kPairRegsSoftmax = 184, kPairRegsEpilogue = 64, kPairRegsOther = 80;
@@ -86,9 +72,7 @@ struct PairLayout {
   static constexpr int kOEmpty = kOUnit + 2;                  // + tile
   static constexpr int kStFull = kOEmpty + 2;                 // + tile
   static constexpr int kStEmpty = kStFull + 2;                // + tile
-  static constexpr int kTok = kStEmpty + 2;                   // + 2 * warp pair + tile
-  static constexpr int kCorr = kTok + 8;                      // + tile: rescale factors ready
-  static constexpr int kDrain = kCorr + 2;
+  static constexpr int kDrain = kStEmpty + 2;
   static constexpr int kUnitFull = kDrain + 1;                // + slot
   static constexpr int kUnitEmpty = kUnitFull + kUnitSlots;   // + slot
   static constexpr int kNumBars = kUnitEmpty + kUnitSlots;
@@ -139,16 +123,12 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     for (int t = 0; t < 2; ++t) {
       ptx::mbar_init(bar(Lay::kSFull + t), 1);
-      // the tile's softmax warps, and the correction warps once they have
-      // rescaled O (the softmax arrives for them at a unit's first step)
-      ptx::mbar_init(bar(Lay::kPFull + t), kCorrectionWG ? 8 : 4);
-      ptx::mbar_init(bar(Lay::kCorr + t), 4);
+      ptx::mbar_init(bar(Lay::kPFull + t), 4);     // the tile's softmax warps
       ptx::mbar_init(bar(Lay::kOUnit + t), 1);
       ptx::mbar_init(bar(Lay::kOEmpty + t), 4);    // epilogue warps
       ptx::mbar_init(bar(Lay::kStFull + t), 4);
       ptx::mbar_init(bar(Lay::kStEmpty + t), 4);
     }
-    for (int i = 0; i < 8; ++i) ptx::mbar_init(bar(Lay::kTok + i), 1);
     ptx::mbar_init(bar(Lay::kDrain), 1);
     for (int i = 0; i < kUnitSlots; ++i) {
       ptx::mbar_init(bar(Lay::kUnitFull + i), 1);
@@ -199,27 +179,6 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const float c = p.scale_log2;
     const uint64_t c2 = ptx::f2_pack(c, c);
     uint32_t g = 0, st_cnt = 0;                    // this tile's key steps, units handed over
-    // Exponential phases of the two tiles take turns on each SM
-    // sub-partition: warp w of tile A and warp w of tile B share one, and a
-    // token passed between them (an mbarrier each way) lets only one of
-    // them run its exponentials at a time.  Tile A goes first.  Both warps
-    // take the same number of turns per unit (the larger step count of the
-    // two tiles; a tile with fewer steps passes the token on unused).
-    const int pair = warp & 3;
-    const uint32_t tok_mine = bar(Lay::kTok + 2 * pair + t);
-    const uint32_t tok_other = bar(Lay::kTok + 2 * pair + (1 - t));
-    uint32_t turns = 0;
-    auto take_turn = [&]() -> bool {
-      if (!kPingPong) return true;
-      const bool r2 = wait_warp(tok_mine, (turns & 1) ^ (t == 0 ? 1u : 0u), ctl);
-      ++turns;
-      return r2;
-    };
-    auto pass_turn = [&]() {
-      if (!kPingPong) return;
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(tok_other);
-    };
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
       const int4 uw = next_unit_warp(k, ok);
@@ -227,12 +186,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const int doc_len = uw.y;
       const int qb = 2 * uw.z + t;
       const int n = tile_steps(qb, doc_len, causal);
-      const int n_turns = max(n, tile_steps(2 * uw.z + (1 - t), doc_len, causal));
-      if (n == 0) {
-        for (int j = 0; j < n_turns && ok; ++j)
-          if ((ok = take_turn())) pass_turn();
-        continue;
-      }
+      if (n == 0) continue;
       float m_used = -INFINITY;   // running maximum in log2 units
       float l = 0.f;              // sum of the weights
       float l_round = 0.f;        // sum of the weights as rounded to bf16
@@ -242,7 +196,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         float s[128];
         {
           uint32_t sa[128];
-          ptx::tmem_ld_2x64(t_s, sa);
+          ptx::tmem_ld_2x64(t_s, sa);     // both halves in flight, one wait
 #pragma unroll
           for (int q = 0; q < 128; ++q) s[q] = __uint_as_float(sa[q]);
         }
@@ -265,24 +219,6 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
         if (j == 0) {
           m_used = m_tile;
-        } else if (kCorrectionWG) {
-          // Lazy rescale: a row whose maximum grew past the threshold takes
-          // the new maximum; its factor 2^(m_used - m_new) (exactly 1 for the
-          // other rows) goes to the correction warps through the last column
-          // of this tile's score buffer, which nothing reads or writes again
-          // before P_t V_j is issued, and they rescale O_t while this warp
-          // computes the weights.
-          const bool need = m_tile > m_used + kRescaleTau;
-          const float m_next = need ? m_tile : m_used;
-          const float alpha = need ? ptx::ex2_approx(m_used - m_next) : 1.f;
-          ptx::tmem_st_x1(t_s + (kBlockN - 1), __float_as_uint(alpha));
-          ptx::tmem_wait_st();
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(bar(Lay::kCorr + t));
-          l *= alpha;
-          l_round *= alpha;
-          m_used = m_next;
         } else {
           // Rescale only rows whose maximum grew past the threshold (warp-wide
           // TMEM access: other rows take part with a factor of exactly 1).
@@ -306,7 +242,6 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         // Weights rounded to bf16 for the P V product; O is divided by the
         // sum of the rounded weights, the log-sum-exp uses the exact sum.
-        if (!(ok = take_turn())) break;
         {
           const float base = m_used == -INFINITY ? 0.f : m_used;
           const uint64_t nb2 = ptx::f2_pack(-base, -base);
@@ -344,17 +279,11 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           l += e0 + e1;
           l_round += (sr[0] + sr[1]) + (sr[2] + sr[3]);
         }
-        pass_turn();
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
-        // At a unit's first step there is nothing to rescale: arrive for the
-        // correction warps as well.
-        if (lane == 0) ptx::mbar_arrive_n(bar(Lay::kPFull + t), kCorrectionWG && j == 0 ? 2u : 1u);
+        if (lane == 0) ptx::mbar_arrive(bar(Lay::kPFull + t));
       }
-      if (!ok) break;
-      for (int j = n; j < n_turns && ok; ++j)
-        if ((ok = take_turn())) pass_turn();
       if (!ok) break;
       if (!(ok = wait_warp(bar(Lay::kStEmpty + t), (st_cnt & 1) ^ 1, ctl))) break;
       ++st_cnt;
@@ -364,98 +293,55 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (lane == 0) ptx::mbar_arrive(bar(Lay::kStFull + t));
     }
   } else if (warp < 12) {
-    // ------------------------------------------------- correction + epilogue
-    // Correction: at every key step after a unit's first, rescale this
-    // warp's 32 rows of O_t by the factors the softmax left in the last
-    // score column (skipped when all are 1), then release P_t V_j.
-    // Epilogue: after a tile's last step, O_t / l_round -> bf16 and the lse.
+    // ------------------------------------------------------------ epilogue
     ptx::regs_decrease<kPairRegsEpilogue>();
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    uint32_t st_cnt[2] = {0, 0}, corr_cnt[2] = {0, 0};
+    uint32_t st_cnt[2] = {0, 0};
     bool ok = true;
-    auto epilogue = [&](int t, int4 uw) -> bool {
-      const int qb = 2 * uw.z + t;
-      const uint32_t cnt = st_cnt[t]++;
-      if (!wait_warp(bar(Lay::kStFull + t), cnt & 1, ctl)) return false;
-      const float lse2 = stats[(2 * t) * kBlockM + r];
-      const float inv_l = stats[(2 * t + 1) * kBlockM + r];
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(Lay::kStEmpty + t));
-      if (!wait_warp(bar(Lay::kOUnit + t), cnt & 1, ctl)) return false;
-      ptx::tc_fence_after();
-      const int row_doc = qb * kBlockM + r;
-      const bool row_ok = row_doc < uw.y;
-      const long long token = static_cast<long long>(uw.x) + row_doc;
-      uint4* orow =
-          reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + (token * H + uw.w) * D);
-      const uint32_t t_o = tmem + lane_off + Lay::kTmemO + t * 128;
-#pragma unroll
-      for (int cc = 0; cc < D / 16; ++cc) {
-        uint32_t o[16];
-        ptx::tmem_ld_x16(t_o + cc * 16, o);
-        if (cc == D / 16 - 1) {
-          // O_t is in registers: the tensor core may overwrite it now.
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(bar(Lay::kOEmpty + t));
-        }
-        uint32_t w[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          w[q] = ptx::pack_bf16x2(__uint_as_float(o[2 * q]) * inv_l,
-                                  __uint_as_float(o[2 * q + 1]) * inv_l);
-        if (row_ok) {
-          orow[cc * 2] = make_uint4(w[0], w[1], w[2], w[3]);
-          orow[cc * 2 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
-        }
-      }
-      if (row_ok)
-        p.lse[static_cast<long long>(uw.w) * p.total_tokens + token] =
-            lse2 * 0.69314718055994530942f;
-      return true;
-    };
-    auto correct = [&](int t) -> bool {
-      if (!wait_warp(bar(Lay::kCorr + t), corr_cnt[t] & 1, ctl)) return false;
-      ++corr_cnt[t];
-      ptx::tc_fence_after();
-      // S_t(j) completed after P_t V_{j-1}, and the softmax saw it complete
-      // before it arrived: O_t is up to date.
-      const float alpha = __uint_as_float(ptx::tmem_ld_x1(tmem + lane_off + t * 128 + (kBlockN - 1)));
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
-        const uint32_t t_o = tmem + lane_off + Lay::kTmemO + t * 128;
+    for (uint32_t k = 0; ok; ++k) {
+      const int4 uw = next_unit_warp(k, ok);
+      if (uw.y < 0) break;
+      for (int t = 0; t < 2 && ok; ++t) {
+        const int qb = 2 * uw.z + t;
+        if (tile_steps(qb, uw.y, causal) == 0) continue;
+        const uint32_t cnt = st_cnt[t]++;
+        if (!(ok = wait_warp(bar(Lay::kStFull + t), cnt & 1, ctl))) break;
+        const float lse2 = stats[(2 * t) * kBlockM + r];
+        const float inv_l = stats[(2 * t + 1) * kBlockM + r];
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar(Lay::kStEmpty + t));
+        if (!(ok = wait_warp(bar(Lay::kOUnit + t), cnt & 1, ctl))) break;
+        ptx::tc_fence_after();
+        const int row_doc = qb * kBlockM + r;
+        const bool row_ok = row_doc < uw.y;
+        const long long token = static_cast<long long>(uw.x) + row_doc;
+        uint4* orow =
+            reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + (token * H + uw.w) * D);
+        const uint32_t t_o = tmem + (static_cast<uint32_t>(wq * 32) << 16) + Lay::kTmemO + t * 128;
 #pragma unroll
         for (int cc = 0; cc < D / 16; ++cc) {
           uint32_t o[16];
           ptx::tmem_ld_x16(t_o + cc * 16, o);
+          if (cc == D / 16 - 1) {
+            // O_t is in registers: the tensor core may overwrite it now.
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar(Lay::kOEmpty + t));
+          }
+          uint32_t w[8];
 #pragma unroll
-          for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          ptx::tmem_st_x16(t_o + cc * 16, o);
+          for (int q = 0; q < 8; ++q)
+            w[q] = ptx::pack_bf16x2(__uint_as_float(o[2 * q]) * inv_l,
+                                    __uint_as_float(o[2 * q + 1]) * inv_l);
+          if (row_ok) {
+            orow[cc * 2] = make_uint4(w[0], w[1], w[2], w[3]);
+            orow[cc * 2 + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+          }
         }
-        ptx::tmem_wait_st();
-      }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(Lay::kPFull + t));
-      return true;
-    };
-    for (uint32_t k = 0; ok; ++k) {
-      const int4 uw = next_unit_warp(k, ok);
-      if (uw.y < 0) break;
-      const int n_t[2] = {tile_steps(2 * uw.z, uw.y, causal),
-                          tile_steps(2 * uw.z + 1, uw.y, causal)};
-      if (!kCorrectionWG) {
-        for (int t = 0; t < 2 && ok; ++t)
-          if (n_t[t] > 0) ok = epilogue(t, uw);
-        continue;
-      }
-      const int n_max = max(n_t[0], n_t[1]);
-      for (int j = 0; j < n_max && ok; ++j) {
-        for (int t = 0; t < 2 && ok; ++t)
-          if (j > 0 && j < n_t[t]) ok = correct(t);
-        for (int t = 0; t < 2 && ok; ++t)
-          if (j == n_t[t] - 1) ok = epilogue(t, uw);
+        if (row_ok)
+          p.lse[static_cast<long long>(uw.w) * p.total_tokens + token] =
+              lse2 * 0.69314718055994530942f;
       }
     }
   } else {

@@ -108,7 +108,7 @@ def test_forced_rescales(d):
     """Scores that grow along the keys (q_i close to a fixed direction u,
     k_j = ramp_j * u) make every row's running maximum rise by more than the
     lazy threshold many times; the result stays exact, and repeated runs are
-    bit-identical (O is rescaled by the correction warps between products)."""
+    bit-identical (O is rescaled between products, never while one runs)."""
     lengths = [700, 1030]
     T, H = sum(lengths), 2
     g = torch.Generator("cpu").manual_seed(21)
