@@ -52,6 +52,12 @@ void timing_mark(int i, cudaStream_t strm) {
   if (cudaEventRecord(g_timing.ev[i], strm) == cudaSuccess && i == 2) g_timing.recorded = true;
 }
 
+// MXFP8 at head dim 128 on the two-query-tile kernel (else the one-tile one).
+#ifndef ATTN_MXFP8_PAIR
+#define ATTN_MXFP8_PAIR 1
+#endif
+constexpr bool kMxfp8Pair = ATTN_MXFP8_PAIR != 0;
+
 constexpr int kMaxDevices = 64;
 constexpr int kScheduleThreads = 1024;
 constexpr int kSortCapacityMax = 16384;                   // 128 KB of keys
@@ -152,12 +158,15 @@ attn_status_t device_info(int* dev_out, DeviceInfo* info) {
         cudaFuncSetAttribute(attn_fwd_kernel<128, kQkNv4>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              FwdLayout<128, kQkNv4>::kBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_pair_kernel<64>,
+        cudaFuncSetAttribute(attn_fwd_pair_kernel<64, kQkBf16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PairLayout<64>::kBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_pair_kernel<128>,
+                             PairLayout<64, kQkBf16>::kBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_pair_kernel<128, kQkBf16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PairLayout<128>::kBytes) != cudaSuccess ||
+                             PairLayout<128, kQkBf16>::kBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_pair_kernel<128, kQkMx8>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PairLayout<128, kQkMx8>::kBytes) != cudaSuccess ||
         cudaFuncSetAttribute(build_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSortCapacityMax * 8) != cudaSuccess)
       return ATTN_ERR_CUDA;
@@ -169,15 +178,16 @@ attn_status_t device_info(int* dev_out, DeviceInfo* info) {
 }
 
 // 3-D map over a [T, H, d] tensor of `elem` bytes per element: box = 128
-// bytes of head dim (the swizzle span) x 1 head x 128 tokens, 128-byte
+// bytes of head dim (the swizzle span) x 1 head x box_rows tokens, 128-byte
 // swizzle, zero fill outside the tensor.
-bool encode_qkv_map(CUtensorMap* m, const void* base, int T, int H, int d, int elem) {
+bool encode_qkv_map(CUtensorMap* m, const void* base, int T, int H, int d, int elem,
+                    int box_rows = kBlockM) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(T)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem,
                                  static_cast<cuuint64_t>(H) * d * elem};
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), 1,
-                             static_cast<cuuint32_t>(kBlockM)};
+                             static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[3] = {1, 1, 1};
   return g_encode(m, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
                   3, const_cast<void*>(base), dims, strides, box, estr,
@@ -282,11 +292,13 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* header = reinterpret_cast<int32_t*>(ws);
 
-  // The block-scaled kernel (MXFP8, d = 128) takes one query tile per unit;
-  // the bf16 kernel two.
+  // bf16 and MXFP8 (d = 128) run the two-query-tile kernel (MXFP8 with
+  // 112-key tiles), NVFP4 (d = 128) the one-tile block-scaled kernel.
   const bool nv4 = dtype == ATTN_NVFP4;
   const bool fp8_kernel = (dtype == ATTN_MXFP8 || nv4) && s.head_dim == 128;
-  const bool pair_kernel = !fp8_kernel;
+  const bool mx8_pair = fp8_kernel && !nv4 && kMxfp8Pair;
+  const bool pair_kernel = !fp8_kernel || mx8_pair;
+  const int kv_rows = mx8_pair ? PairLayout<128, kQkMx8>::kBN : kBlockN;
   timing_mark(0, strm);
   // 1. schedule (validates cu_seqlens, writes the work list and its length)
   const int64_t cap = sort_capacity_for(wl.max_entries);
@@ -383,10 +395,12 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
         !encode_fp4_map(&tk, qk_src[1], s.total_tokens, s.num_heads, s.head_dim))
       return ATTN_ERR_CUDA;
   } else if (!encode_qkv_map(&tq, qk_src[0], s.total_tokens, s.num_heads, s.head_dim, qk_elem) ||
-             !encode_qkv_map(&tk, qk_src[1], s.total_tokens, s.num_heads, s.head_dim, qk_elem)) {
+             !encode_qkv_map(&tk, qk_src[1], s.total_tokens, s.num_heads, s.head_dim, qk_elem,
+                             kv_rows)) {
     return ATTN_ERR_CUDA;
   }
-  if (!encode_qkv_map(&tv, v, s.total_tokens, s.num_heads, s.head_dim, 2)) return ATTN_ERR_CUDA;
+  if (!encode_qkv_map(&tv, v, s.total_tokens, s.num_heads, s.head_dim, 2, kv_rows))
+    return ATTN_ERR_CUDA;
   FwdParams fp;
   fp.out = out;
   fp.lse = lse;
@@ -420,15 +434,18 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
   if (fp8_kernel && nv4) {
     cfg.dynamicSmemBytes = FwdLayout<128, kQkNv4>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, kQkNv4>, tq, tk, tv, fp);
+  } else if (mx8_pair) {
+    cfg.dynamicSmemBytes = PairLayout<128, kQkMx8>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<128, kQkMx8>, tq, tk, tv, fp);
   } else if (fp8_kernel) {
     cfg.dynamicSmemBytes = FwdLayout<128, kQkMx8>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, kQkMx8>, tq, tk, tv, fp);
   } else if (s.head_dim == 128) {
-    cfg.dynamicSmemBytes = PairLayout<128>::kBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<128>, tq, tk, tv, fp);
+    cfg.dynamicSmemBytes = PairLayout<128, kQkBf16>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<128, kQkBf16>, tq, tk, tv, fp);
   } else {
-    cfg.dynamicSmemBytes = PairLayout<64>::kBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<64>, tq, tk, tv, fp);
+    cfg.dynamicSmemBytes = PairLayout<64, kQkBf16>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<64, kQkBf16>, tq, tk, tv, fp);
   }
   timing_mark(2, strm);
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

@@ -50,18 +50,35 @@ static_assert(2 * kPairRegsSoftmax + kPairRegsEpilogue + kPairRegsOther == 4 * 1
               "register split must use exactly the registers the CTA is launched with");
 constexpr int kPairUnitConsumers = 1 + 8 + 4;   // MMA thread + softmax warps + epilogue warps
 
-template <int D>
+// Score operand format kQk (attn_fwd_sm100.cuh): bf16, or MXFP8 (E4M3 codes
+// with one E8M0 scale per 32 elements; head dim 128).  MXFP8 uses key tiles
+// of 112: the score products are then 112 columns wide, which leaves the
+// last 16 columns of each tile's score buffer for the scale factors (Q's
+// of each tile, and two buffers of the K tile's).
+template <int D, int kQk>
 struct PairLayout {
+  static constexpr bool kFp8 = kQk == kQkMx8;
+  static_assert(kQk == kQkBf16 || kQk == kQkMx8, "pair kernel: bf16 or MXFP8 score operands");
   static_assert(D == 64 || D == 128, "head dim 64 or 128");
-  static constexpr int kChunks = D / 64;                      // 128-byte chunks per row
-  static constexpr int kChunkBytes = kBlockM * 128;           // 128 rows x 128 bytes
-  static constexpr int kTileBytes = kChunks * kChunkBytes;    // one Q, K or V tile
+  static_assert(!kFp8 || D == 128, "MXFP8 pair kernel: head dim 128");
+  static constexpr int kBN = kFp8 ? 112 : 128;                // keys per K/V tile
+  static constexpr int kChunks = D / 64;                      // 128-byte chunks of a bf16 row
+  static constexpr int kQkChunks = kFp8 ? 1 : kChunks;        // ... of a Q or K row
+  static constexpr int kQTileBytes = kQkChunks * kBlockM * 128;
+  static constexpr int kKTileBytes = kQkChunks * kBN * 128;
+  static constexpr int kVChunkBytes = kBN * 128;
+  static constexpr int kVTileBytes = kChunks * kVChunkBytes;
+  static constexpr int kSfBytes = kFp8 ? 512 : 0;             // scale block of a Q or K tile
+  static constexpr int kSlotRaw = kVTileBytes > kKTileBytes + kSfBytes ? kVTileBytes
+                                                                       : kKTileBytes + kSfBytes;
+  static constexpr int kSlotBytes = (kSlotRaw + 1023) / 1024 * 1024;   // a K (+ scales) or V tile
   static constexpr int kQOff = 0;                             // Q_A, then Q_B
-  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kSfaOff = 2 * kQTileBytes;             // MXFP8: Q_A's, Q_B's scale blocks
+  static constexpr int kRingOff = (kSfaOff + 2 * kSfBytes + 1023) / 1024 * 1024;
   static constexpr int kReserve = 3072;                       // stats, barriers, unit ring
-  static constexpr int kStagesFit = (232448 - kRingOff - kReserve) / kTileBytes;
+  static constexpr int kStagesFit = (232448 - kRingOff - kReserve) / kSlotBytes;
   static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
-  static constexpr int kStatsOff = kRingOff + kStages * kTileBytes;   // float [tile][2][128]
+  static constexpr int kStatsOff = kRingOff + kStages * kSlotBytes;   // float [tile][2][128]
   static constexpr int kBarOff = kStatsOff + 2 * 2 * kBlockM * 4;
   static constexpr int kQFull = 0, kQEmpty = 1;
   static constexpr int kKVFull = 2;                           // + stage
@@ -82,23 +99,29 @@ struct PairLayout {
   static_assert(kStages >= 3, "too few K/V stages");
   static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
   static_assert(kBytes - kStatsOff <= kReserve, "reserve too small");
+  static_assert(kSlotBytes % 1024 == 0 && kVChunkBytes % 1024 == 0, "swizzle alignment");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemO = 256;                     // + 128 * tile
+  // MXFP8 scale factors in the unused columns 112..127 of the score buffers:
+  // Q_t's at 128 t + 112, the K tiles' (two buffers) at 116 and 120.
+  static constexpr uint32_t kTmemSfa = 112, kTmemSfb = 116;
 };
 
-// Key steps of query tile qb of a document of doc_len tokens (0 if the tile
-// starts past the document's end).
-__device__ __forceinline__ int tile_steps(int qb, int doc_len, int causal) {
+// Key steps of query tile qb (128 rows) of a document of doc_len tokens with
+// key tiles of bn keys (0 if the tile starts past the document's end).
+__device__ __forceinline__ int tile_steps(int qb, int doc_len, int causal, int bn = kBlockN) {
   if (qb * kBlockM >= doc_len) return 0;
-  const int kv = (doc_len + kBlockN - 1) / kBlockN;
-  return causal ? min(qb + 1, kv) : kv;
+  const int last = causal ? min(doc_len, (qb + 1) * kBlockM) : doc_len;   // keys seen
+  return (last + bn - 1) / bn;
 }
 
-template <int D>
+template <int D, int kQk>
 __global__ void __launch_bounds__(kPairThreads, 1)
 attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Lay = PairLayout<D>;
+  using Lay = PairLayout<D, kQk>;
+  constexpr bool kFp8 = Lay::kFp8;
+  constexpr int BN = Lay::kBN;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = ptx::smem_addr(smem);
   if ((sbase & 1023u) != 0) {
@@ -185,7 +208,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (uw.y < 0) break;
       const int doc_len = uw.y;
       const int qb = 2 * uw.z + t;
-      const int n = tile_steps(qb, doc_len, causal);
+      const int n = tile_steps(qb, doc_len, causal, BN);
       if (n == 0) continue;
       float m_used = -INFINITY;   // running maximum in log2 units
       float l = 0.f;              // sum of the weights
@@ -200,19 +223,22 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
           for (int q = 0; q < 128; ++q) s[q] = __uint_as_float(sa[q]);
         }
-        const bool diag = causal && j == qb;
-        if (diag || (j + 1) * kBlockN > doc_len) {
-          int limit = doc_len - j * kBlockN;
-          if (diag) limit = min(limit, r + 1);
+        // Keys past the document's end or (causal) past this row: -inf.  A
+        // tile needs masking if it reaches past the document or, causal,
+        // past the tile's first row.
+        const bool diag = causal && (j + 1) * BN - 1 > qb * kBlockM;
+        if (diag || (j + 1) * BN > doc_len) {
+          int limit = doc_len - j * BN;
+          if (diag) limit = min(limit, qb * kBlockM + r + 1 - j * BN);
 #pragma unroll
-          for (int q = 0; q < 128; ++q)
+          for (int q = 0; q < BN; ++q)
             if (q >= limit) s[q] = -INFINITY;
         }
         float mx[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) mx[a] = fmaxf(s[2 * a], s[2 * a + 1]);
 #pragma unroll
-        for (int q = 16; q < 128; q += 16)
+        for (int q = 16; q < BN; q += 16)
 #pragma unroll
           for (int a = 0; a < 8; ++a) mx[a] = ptx::fmax3(mx[a], s[q + 2 * a], s[q + 2 * a + 1]);
         const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
@@ -251,12 +277,14 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           for (int a = 0; a < 2; ++a) se[a] = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
           for (int a = 0; a < 4; ++a) sr[a] = 0.f;
+          // P in chunks of kPk key pairs (one TMEM store each)
+          constexpr int kPk = BN % 32 == 0 ? 16 : 8;
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t pk[16];
+          for (int ch = 0; ch < BN / (2 * kPk); ++ch) {
+            uint32_t pk[kPk];
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk) {
-              const int q = ch * 16 + kk;
+            for (int kk = 0; kk < kPk; ++kk) {
+              const int q = ch * kPk + kk;
               const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[2 * q], s[2 * q + 1]), c2, nb2);
               float x0, x1, p0, p1;
               ptx::f2_unpack(x, x0, x1);
@@ -272,7 +300,10 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
               sr[(kk & 1) * 2] = ptx::add_bf16_lo(sr[(kk & 1) * 2], pk[kk]);
               sr[(kk & 1) * 2 + 1] = ptx::add_bf16_hi(sr[(kk & 1) * 2 + 1], pk[kk]);
             }
-            ptx::tmem_st_x16(t_s + ch * 16, pk);
+            if constexpr (kPk == 16)
+              ptx::tmem_st_x16(t_s + ch * 16, pk);
+            else
+              ptx::tmem_st_x8(t_s + ch * 8, pk);
           }
           float e0, e1;
           ptx::f2_unpack(ptx::f2_add(se[0], se[1]), e0, e1);
@@ -304,7 +335,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (uw.y < 0) break;
       for (int t = 0; t < 2 && ok; ++t) {
         const int qb = 2 * uw.z + t;
-        if (tile_steps(qb, uw.y, causal) == 0) continue;
+        if (tile_steps(qb, uw.y, causal, BN) == 0) continue;
         const uint32_t cnt = st_cnt[t]++;
         if (!(ok = wait_warp(bar(Lay::kStFull + t), cnt & 1, ctl))) break;
         const float lse2 = stats[(2 * t) * kBlockM + r];
@@ -352,15 +383,43 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       int* counter = const_cast<int*>(p.ws_header) + kWsUnitCounterOffset / 4;
       uint32_t q_it = 0, kv_it = 0;
       bool ok = true;
-      auto load_kv = [&](int head, int row0, const CUtensorMap* tm) -> bool {
+      // Scale block of the 128 rows from row0 (MXFP8): lane m0 writes rows
+      // m0 + 32 c, c = 0..3, as 16 bytes at offset 16 m0 (the layout
+      // tcgen05.cp replicates); rows past `rows` or the tensor get 0.
+      auto stage_scales = [&](const uint32_t* scales, int head, int row0, int rows, int off) {
+        uint32_t wv[4];
+#pragma unroll
+        for (int cq = 0; cq < 4; ++cq) {
+          const int rr = lane + 32 * cq;
+          const int tok = row0 + rr;
+          wv[cq] = rr < rows && tok < p.total_tokens
+                       ? scales[static_cast<long long>(tok) * H + head] : 0u;
+        }
+        *reinterpret_cast<uint4*>(smem + off + 16 * lane) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      };
+      // One K (kind 0) or V (kind 1) tile into the next ring slot.
+      auto load_kv = [&](int head, int row0, int kind) -> bool {
         const uint32_t s = kv_it % Lay::kStages;
         if (!wait_warp(bar(Lay::kKVEmpty + s), ((kv_it / Lay::kStages) & 1) ^ 1, ctl)) return false;
+        if (kFp8 && kind == 0) {
+          stage_scales(p.k_scales, head, row0, BN,
+                       Lay::kRingOff + s * Lay::kSlotBytes + Lay::kKTileBytes);
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
         if (lane == 0) {
-          const uint32_t slot = sbase + Lay::kRingOff + s * Lay::kTileBytes;
-          ptx::mbar_arrive_expect_tx(bar(Lay::kKVFull + s), Lay::kTileBytes);
-          for (int cq = 0; cq < Lay::kChunks; ++cq)
-            ptx::tma_load_3d(slot + cq * Lay::kChunkBytes, tm, bar(Lay::kKVFull + s), cq * 64,
-                             head, row0);
+          const uint32_t slot = sbase + Lay::kRingOff + s * Lay::kSlotBytes;
+          if (kind == 0) {
+            ptx::mbar_arrive_expect_tx(bar(Lay::kKVFull + s), Lay::kKTileBytes);
+            for (int cq = 0; cq < Lay::kQkChunks; ++cq)
+              ptx::tma_load_3d(slot + cq * BN * 128, &tm_k, bar(Lay::kKVFull + s),
+                               cq * (kFp8 ? 128 : 64), head, row0);
+          } else {
+            ptx::mbar_arrive_expect_tx(bar(Lay::kKVFull + s), Lay::kVTileBytes);
+            for (int cq = 0; cq < Lay::kChunks; ++cq)
+              ptx::tma_load_3d(slot + cq * Lay::kVChunkBytes, &tm_v, bar(Lay::kKVFull + s),
+                               cq * 64, head, row0);
+          }
         }
         __syncwarp();
         ++kv_it;
@@ -404,24 +463,32 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         __syncwarp();
         if (uw.y < 0) break;
-        const int n_max =
-            max(tile_steps(2 * uw.z, uw.y, causal), tile_steps(2 * uw.z + 1, uw.y, causal));
+        const int n_max = max(tile_steps(2 * uw.z, uw.y, causal, BN),
+                              tile_steps(2 * uw.z + 1, uw.y, causal, BN));
         if (!(ok = wait_warp(bar(Lay::kQEmpty), (q_it & 1) ^ 1, ctl))) break;
         const int qrow0 = uw.x + 2 * kBlockM * uw.z;
-        if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(bar(Lay::kQFull), 2 * Lay::kTileBytes);
+        if constexpr (kFp8) {
           for (int t = 0; t < 2; ++t)
-            for (int cq = 0; cq < Lay::kChunks; ++cq)
-              ptx::tma_load_3d(sbase + Lay::kQOff + t * Lay::kTileBytes + cq * Lay::kChunkBytes,
-                               &tm_q, bar(Lay::kQFull), cq * 64, uw.w, qrow0 + t * kBlockM);
+            stage_scales(p.q_scales, uw.w, qrow0 + t * kBlockM, kBlockM,
+                         Lay::kSfaOff + t * Lay::kSfBytes);
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(bar(Lay::kQFull), 2 * Lay::kQTileBytes);
+          for (int t = 0; t < 2; ++t)
+            for (int cq = 0; cq < Lay::kQkChunks; ++cq)
+              ptx::tma_load_3d(sbase + Lay::kQOff + t * Lay::kQTileBytes + cq * kBlockM * 128,
+                               &tm_q, bar(Lay::kQFull), cq * (kFp8 ? 128 : 64), uw.w,
+                               qrow0 + t * kBlockM);
         }
         __syncwarp();
         ++q_it;
         // ring order = consumption order: K_0, then V_j, K_{j+1}
-        if (!(ok = load_kv(uw.w, uw.x, &tm_k))) break;
+        if (!(ok = load_kv(uw.w, uw.x, 0))) break;
         for (int j = 0; ok && j < n_max; ++j) {
-          if (!(ok = load_kv(uw.w, uw.x + kBlockN * j, &tm_v))) break;
-          if (j + 1 < n_max && !(ok = load_kv(uw.w, uw.x + kBlockN * (j + 1), &tm_k))) break;
+          if (!(ok = load_kv(uw.w, uw.x + BN * j, 1))) break;
+          if (j + 1 < n_max && !(ok = load_kv(uw.w, uw.x + BN * (j + 1), 0))) break;
         }
       }
       if (!ok && lane == 0) {
@@ -436,16 +503,17 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
     } else if (warp == kWarpMma && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t kIdescS = ptx::idesc_bf16(kBlockM, kBlockN, 0);
+      constexpr uint32_t kIdescS = ptx::idesc_bf16(kBlockM, BN, 0);
       constexpr uint32_t kIdescO = ptx::idesc_bf16(kBlockM, D, 1);
       constexpr uint32_t kDescHi = ptx::sdesc_hi_sw128(1024);
       const uint32_t q_lo = ptx::sdesc_lo(sbase + Lay::kQOff, 16);
       const uint32_t ring_lo = ptx::sdesc_lo(sbase + Lay::kRingOff, 16);
-      const uint32_t v_lbo = static_cast<uint32_t>(Lay::kChunkBytes - 16) >> 4 << 16;
+      const uint32_t v_lbo = static_cast<uint32_t>(Lay::kVChunkBytes - 16) >> 4 << 16;
       uint32_t q_ph = 0;
       uint32_t g[2] = {0, 0};          // key steps of each tile so far
       uint32_t oe_cnt[2] = {0, 0};     // units of each tile so far
       uint32_t cur = 0, cur_ph = 0;    // ring cursor (stage, phase)
+      uint32_t k_cnt = 0;              // K tiles taken (MXFP8: scale buffer k_cnt & 1)
       bool ok = true;
       auto take = [&](uint32_t& st) -> bool {
         st = cur;
@@ -456,23 +524,53 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         return r2;
       };
+      // The next K tile; MXFP8: its scale block into the next TMEM buffer
+      // (the products that read that buffer two K tiles ago were issued
+      // before, and the tensor pipe keeps issue order).
+      auto take_k = [&](uint32_t& st) -> bool {
+        if (!take(st)) return false;
+        if constexpr (kFp8) {
+          ptx::tc_fence_after();
+          tmem_cp_32x128b_x4(tmem + Lay::kTmemSfb + 4 * (k_cnt & 1),
+                             sf_copy_desc(sbase + Lay::kRingOff + st * Lay::kSlotBytes +
+                                          Lay::kKTileBytes));
+        }
+        ++k_cnt;
+        return true;
+      };
       // S_t = Q_t K^T with K in ring stage st
       auto score = [&](int t, uint32_t st, bool commit = true) {
-        const uint32_t a_lo = q_lo + ((t * Lay::kTileBytes) >> 4);
-        const uint32_t b_lo = ring_lo + st * (Lay::kTileBytes >> 4);
+        const uint32_t a_lo = q_lo + ((t * Lay::kQTileBytes) >> 4);
+        const uint32_t b_lo = ring_lo + st * (Lay::kSlotBytes >> 4);
+        if constexpr (kFp8) {
+          // block-scaled E4M3: four K = 32 products, scale byte kk of each
+          // row's word
+          const uint32_t sfa = tmem + t * 128 + Lay::kTmemSfa;
+          const uint32_t sfb = tmem + Lay::kTmemSfb + 4 * ((k_cnt - 1) & 1);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * Lay::kChunkBytes + (kk & 3) * 32) >> 4;
-          ptx::mma_f16_ss(tmem + t * 128, ptx::sdesc_join(a_lo + off, kDescHi),
-                          ptx::sdesc_join(b_lo + off, kDescHi), kIdescS, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 32; ++kk) {
+            const uint32_t off = (kk * 32) >> 4;
+            mma_mxf8_ss(tmem + t * 128, ptx::sdesc_join(a_lo + off, kDescHi),
+                        ptx::sdesc_join(b_lo + off, kDescHi), idesc_mxf8(kk, BN),
+                        (static_cast<uint32_t>(kk) << 30) | sfa,
+                        (static_cast<uint32_t>(kk) << 30) | sfb, kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * BN * 128 + (kk & 3) * 32) >> 4;
+            const uint32_t a_off = ((kk >> 2) * kBlockM * 128 + (kk & 3) * 32) >> 4;
+            ptx::mma_f16_ss(tmem + t * 128, ptx::sdesc_join(a_lo + a_off, kDescHi),
+                            ptx::sdesc_join(b_lo + off, kDescHi), kIdescS, kk > 0 ? 1u : 0u);
+          }
         }
         if (commit) ptx::mma_commit(bar(Lay::kSFull + t));
       };
       // O_t += P_t V with V in ring stage st
       auto pv = [&](int t, int j, uint32_t st) {
-        const uint32_t b_lo = ring_lo + st * (Lay::kTileBytes >> 4) + v_lbo;
+        const uint32_t b_lo = ring_lo + st * (Lay::kSlotBytes >> 4) + v_lbo;
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk)
+        for (int kk = 0; kk < BN / 16; ++kk)
           ptx::mma_f16_ts(tmem + Lay::kTmemO + t * 128, tmem + t * 128 + kk * 8,
                           ptx::sdesc_join(b_lo + kk * (2048 >> 4), kDescHi), kIdescO,
                           (j == 0 && kk == 0) ? 0u : 1u);
@@ -483,13 +581,19 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const int4 uw = unit_ring[uslot];
         ptx::mbar_arrive(bar(Lay::kUnitEmpty + uslot));
         if (uw.y < 0) break;
-        const int n_t[2] = {tile_steps(2 * uw.z, uw.y, causal), tile_steps(2 * uw.z + 1, uw.y, causal)};
+        const int n_t[2] = {tile_steps(2 * uw.z, uw.y, causal, BN),
+                            tile_steps(2 * uw.z + 1, uw.y, causal, BN)};
         const int n_max = max(n_t[0], n_t[1]);
         if (!(ok = wait_one(bar(Lay::kQFull), q_ph, ctl))) break;
         q_ph ^= 1;
         ptx::tc_fence_after();
+        if constexpr (kFp8) {
+          for (int t = 0; t < 2; ++t)
+            tmem_cp_32x128b_x4(tmem + t * 128 + Lay::kTmemSfa,
+                               sf_copy_desc(sbase + Lay::kSfaOff + t * Lay::kSfBytes));
+        }
         uint32_t st_k, st_v;
-        if (!(ok = take(st_k))) break;
+        if (!(ok = take_k(st_k))) break;
         for (int t = 0; t < 2; ++t)
           if (n_t[t] > 0) score(t, st_k, !(kFaultDropFirstScoreCommit && k == 0 && t == 0));
         ptx::mma_commit(bar(Lay::kKVEmpty + st_k));
@@ -510,7 +614,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             ++g[t];
             if (j + 1 < n_t[t]) {
               if (!k_taken) {
-                if (!(ok = take(st_k))) break;
+                if (!(ok = take_k(st_k))) break;
                 k_taken = true;
               }
               score(t, st_k);
@@ -519,7 +623,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           if (!ok) break;
           ptx::mma_commit(bar(Lay::kKVEmpty + st_v));
           if (j + 1 < n_max) {
-            if (!k_taken && !(ok = take(st_k))) break;   // unreachable: n_max's tile needs it
+            if (!k_taken && !(ok = take_k(st_k))) break;   // unreachable: n_max's tile needs it
             ptx::mma_commit(bar(Lay::kKVEmpty + st_k));
             if (j + 2 == n_max) ptx::mma_commit(bar(Lay::kQEmpty));
           }

@@ -268,12 +268,12 @@ __device__ __forceinline__ uint64_t sf_copy_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor for the block-scaled E4M3 x E4M3 product (fp32
-// accumulate, E8M0 scales, M = N = 128, K = 32); sf_id picks the scale byte
-// (the 32-element block) inside each 32-bit scale column.
-__host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t sf_id) {
+// accumulate, E8M0 scales, M = 128, N = n, K = 32); sf_id picks the scale
+// byte (the 32-element block) inside each 32-bit scale column.
+__host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t sf_id, int n = kBlockN) {
   return (sf_id << 4)                         // B scale id
          | (0u << 7) | (0u << 10)             // A, B format: E4M3
-         | (static_cast<uint32_t>(kBlockN >> 3) << 17)
+         | (static_cast<uint32_t>(n >> 3) << 17)
          | (1u << 23)                         // scale format: E8M0
          | (static_cast<uint32_t>(kBlockM >> 4) << 24)
          | (sf_id << 29);                     // A scale id
