@@ -63,7 +63,8 @@ INCOHERENT_SECTION_MARK = b"\n// " + b"=" * 75 + b"\n// Incoherent processing"
 # The CUDA sources each measured kernel is built and launched from, and the
 # marker where that part's share of attn_api.cu ends.
 FWD_SOURCES = ["attn_api.cu", "attn_fwd_pair_sm100.cuh", "attn_fwd_sm100.cuh", "common.cuh",
-               "ptx.cuh", "quant_mxfp8.cuh", "schedule.cuh", "tmem_ops.cuh"]
+               "incoherent.cuh", "ptx.cuh", "quant_mxfp8.cuh", "quant_nvfp4.cuh", "schedule.cuh",
+               "tmem_ops.cuh"]
 PART_SOURCES = {
     "fwd": (FWD_SOURCES, BWD_SECTION_MARK),
     "bwd": (FWD_SOURCES + ["attn_bwd_sm100.cuh"], INCOHERENT_SECTION_MARK),

@@ -324,19 +324,21 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
     for (int i = 0; i < 3; ++i) {
       const bool use_codes = fp8_kernel && i < 2;
       jobs.t[i].x = static_cast<const uint4*>(src[i]);
-      jobs.t[i].codes = use_codes ? reinterpret_cast<uint4*>(ws + wl.codes_off[i]) : nullptr;
+      jobs.t[i].codes = use_codes ? reinterpret_cast<uint2*>(ws + wl.codes_off[i]) : nullptr;
       jobs.t[i].scales = use_codes ? ws + wl.scales_off[i] : nullptr;
       jobs.t[i].deq = use_codes ? nullptr : reinterpret_cast<uint4*>(ws + wl.deq_off[i]);
       jobs.t[i].rotate = i < 2 ? 1 : 0;
     }
-    const long long qgrid = (jobs.rows + 127) / 128;
+    // D / 8 lanes per row, 256 threads per block
+    const long long rows_per_block = 256 / (s.head_dim / 8);
+    const long long qgrid = (jobs.rows + rows_per_block - 1) / rows_per_block;
     if (qgrid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     if (s.head_dim == 128)
       quantize_mxfp8_incoherent_qkv_kernel<128>
-          <<<dim3(static_cast<unsigned>(qgrid), 3), 128, 0, strm>>>(jobs, signs);
+          <<<dim3(static_cast<unsigned>(qgrid), 3), 256, 0, strm>>>(jobs, signs);
     else
       quantize_mxfp8_incoherent_qkv_kernel<64>
-          <<<dim3(static_cast<unsigned>(qgrid), 3), 128, 0, strm>>>(jobs, signs);
+          <<<dim3(static_cast<unsigned>(qgrid), 3), 256, 0, strm>>>(jobs, signs);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     for (int i = 0; i < 2; ++i) qk_src[i] = ws + (fp8_kernel ? wl.codes_off[i] : wl.deq_off[i]);
     v = ws + wl.deq_off[2];
@@ -782,15 +784,16 @@ extern "C" attn_status_t attn_quantize_mxfp8_rotated(const void* x, const float*
     return ATTN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u) != 0)
     return ATTN_ERR_ALIGNMENT;
-  const long long grid = (rows + 127) / 128;
+  const long long rows_per_block = 256 / (cols / 8);
+  const long long grid = (rows + rows_per_block - 1) / rows_per_block;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   if (cols == 128)
-    quantize_mxfp8_rotated_kernel<128><<<static_cast<unsigned>(grid), 128, 0, strm>>>(
-        static_cast<const uint4*>(x), signs, reinterpret_cast<uint4*>(codes), scales, rows);
+    quantize_mxfp8_rotated_kernel<128><<<static_cast<unsigned>(grid), 256, 0, strm>>>(
+        static_cast<const uint4*>(x), signs, reinterpret_cast<uint2*>(codes), scales, rows);
   else
-    quantize_mxfp8_rotated_kernel<64><<<static_cast<unsigned>(grid), 128, 0, strm>>>(
-        static_cast<const uint4*>(x), signs, reinterpret_cast<uint4*>(codes), scales, rows);
+    quantize_mxfp8_rotated_kernel<64><<<static_cast<unsigned>(grid), 256, 0, strm>>>(
+        static_cast<const uint4*>(x), signs, reinterpret_cast<uint2*>(codes), scales, rows);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -92,23 +92,6 @@ constexpr int kHalfKeys = kBlockN / 2;
 constexpr int kUnitSlots = 4;
 constexpr int kUnitConsumers = 1 + kSoftmaxWarps + 4;   // MMA thread + softmax + epilogue warps
 
-// Exponentials: most run on the MUFU unit (ex2.approx); pairs of keys with
-// index k % period == period - 1 run on the FMA pipe instead, as 2^x =
-// 2^floor(x) * p(frac(x)) with the polynomial below (0 = MUFU only).  The MUFU
-// unit alone cannot keep up with the tensor core (16 exponentials per SM and
-// cycle against 128 x 128 scores per 128 x 128 x D product pair).
-#ifndef ATTN_POLY_PAIR_PERIOD
-#define ATTN_POLY_PAIR_PERIOD 0
-#endif
-constexpr int kPolyPairPeriod = ATTN_POLY_PAIR_PERIOD;
-
-
-// 2^f on [0, 1): 1 + f (c1 + f (c2 + f c3)), a minimax fit of the relative
-// error (max 8.6e-5), found by linear programming over a dense grid of
-// [0, 1) with the constant term fixed at 1, so p(0) = 1 exactly.
-constexpr float kExp2C1 = 6.951168180e-01f;
-constexpr float kExp2C2 = 2.276448607e-01f;
-constexpr float kExp2C3 = 7.706713676e-02f;
 
 // Operand format of the score product Q K^T: bf16, MXFP8 (E4M3 codes, one
 // E8M0 scale per 32 elements) or NVFP4 (E2M1 codes two per byte, one
@@ -238,27 +221,6 @@ __device__ __forceinline__ UnitInfo decode_unit(int4 w, int causal) {
   r.kv_tiles = (w.y + kBlockN - 1) / kBlockN;
   r.n = causal ? min(w.z + 1, r.kv_tiles) : r.kv_tiles;
   return r;
-}
-
-// 2^x for a pair of x <= 8 on the FMA pipe.  x = j + f with j = floor(x)
-// (taken from adding 1.5 * 2^23 rounded down, which leaves j in the low
-// mantissa bits), 2^f from the polynomial, and j added to the exponent
-// field.  x is clamped at -127 first, where the result is exactly +0 (the
-// exponent field of p(0) = 1 cancels), so masked scores (-inf) give 0.
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
-  const uint64_t x = ptx::f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
-  const float kMagic = 12582912.f;   // 1.5 * 2^23
-  const uint64_t t = ptx::f2_add_rm(x, ptx::f2_pack(kMagic, kMagic));
-  const uint64_t jf = ptx::f2_add(t, ptx::f2_pack(-kMagic, -kMagic));
-  const uint64_t f = ptx::f2_fma(jf, ptx::f2_pack(-1.f, -1.f), x);
-  uint64_t q = ptx::f2_fma(ptx::f2_pack(kExp2C3, kExp2C3), f, ptx::f2_pack(kExp2C2, kExp2C2));
-  q = ptx::f2_fma(q, f, ptx::f2_pack(kExp2C1, kExp2C1));
-  q = ptx::f2_fma(q, f, ptx::f2_pack(1.f, 1.f));
-  float q0, q1, t0, t1;
-  ptx::f2_unpack(q, q0, q1);
-  ptx::f2_unpack(t, t0, t1);
-  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 // Shared-memory descriptor of a 32-row x 16-byte block of E8M0 scales for
@@ -519,13 +481,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[2 * q], s[2 * q + 1]), c2, nb2);
             float x0, x1, p0, p1;
             ptx::f2_unpack(x, x0, x1);
-            if (kPolyPairPeriod > 0 &&
-                q % (kPolyPairPeriod > 0 ? kPolyPairPeriod : 1) == kPolyPairPeriod - 1) {
-              exp2_poly_pair(x0, x1, p0, p1);
-            } else {
-              p0 = ptx::ex2_approx(x0);
-              p1 = ptx::ex2_approx(x1);
-            }
+            p0 = ptx::ex2_approx(x0);
+            p1 = ptx::ex2_approx(x1);
             pk[q] = ptx::pack_bf16x2(p0, p1);
             se[q & 1] = ptx::f2_add(se[q & 1], ptx::f2_pack(p0, p1));
             sr[(q & 1) * 2] = ptx::add_bf16_lo(sr[(q & 1) * 2], pk[q]);

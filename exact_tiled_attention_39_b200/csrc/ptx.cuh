@@ -226,13 +226,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// a + b rounded toward minus infinity.
-__device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
 // acc + (bf16 in the low / high half of w), computed in fp32.
 __device__ __forceinline__ float add_bf16_lo(float acc, uint32_t w) {
   float d;
