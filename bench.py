@@ -267,12 +267,13 @@ def kernel_name_for(dtype_name: str) -> str:
 
 
 def measure_workload(A, name, steps, warmup, dev, stream, pg, clk):
-    """Time one workload: `steps` back-to-back attn_fwd calls (device events,
-    barrier + synchronize on both sides, max over ranks), then the attention
-    kernel alone (CUDA events the library records on the launching stream
-    around that kernel; median over at least KERNEL_TIMING_LAUNCHES launches
-    and KERNEL_TIMING_MIN_S of device time).  Returns the figures and the
-    device tensors for the end-to-end leg."""
+    """Time one workload: after `warmup` untimed calls, the attention kernel
+    alone (CUDA events the library records on the launching stream around
+    that kernel; median over at least KERNEL_TIMING_LAUNCHES launches and
+    KERNEL_TIMING_MIN_S of device time), then `steps` back-to-back attn_fwd
+    calls (device events, barrier + synchronize on both sides, max over
+    ranks).  Returns the figures and the device tensors for the end-to-end
+    leg."""
     w = workloads.get(name)
     inp = workloads.make_inputs(w)
     T, H, d = inp["q"].shape
@@ -302,17 +303,10 @@ def measure_workload(A, name, steps, warmup, dev, stream, pg, clk):
     torch.cuda.synchronize(dev)
     assert A.attn_get_device_error(ws) == 0, f"device error during warm-up ({name})"
 
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize(dev)
     with clk:
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for _ in range(steps):
-            step()
-        t1.record(stream)
-        torch.cuda.synchronize(dev)
+        # The attention kernel alone, before the timed steps: it also brings
+        # the GPU from idle (input generation) to its steady clocks, so the
+        # timed steps below measure steady-state throughput.
         A.attn_timing_enable(True)
         per, pre = [], []
         while len(per) < KERNEL_TIMING_LAUNCHES or sum(per) < 1e3 * KERNEL_TIMING_MIN_S:
@@ -323,6 +317,17 @@ def measure_workload(A, name, steps, warmup, dev, stream, pg, clk):
             if len(per) >= 20000:
                 break
         A.attn_timing_enable(False)
+        # ---- device-timed region: `steps` back-to-back steps, barrier +
+        # synchronize on both sides
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
         torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()

@@ -49,13 +49,6 @@ constexpr uint32_t kPairRegsSoftmax = 184, kPairRegsEpilogue = 64, kPairRegsOthe
 static_assert(2 * kPairRegsSoftmax + kPairRegsEpilogue + kPairRegsOther == 4 * 128,
               "register split must use exactly the registers the CTA is launched with");
 constexpr int kPairUnitConsumers = 1 + 8 + 4;   // MMA thread + softmax warps + epilogue warps
-// P of a key step is handed to the tensor core in two parts, keys
-// [0, kPLoKeys) and the rest, so the first part's products overlap the
-// forming of the second part's weights.
-#ifndef ATTN_P_LO_KEYS
-#define ATTN_P_LO_KEYS 64
-#endif
-constexpr int kPLoKeys = ATTN_P_LO_KEYS;   // 0: one hand-off per step
 
 // Score operand format kQk (attn_fwd_sm100.cuh): bf16, or MXFP8 (E4M3 codes
 // with one E8M0 scale per 32 elements; head dim 128).  MXFP8 uses key tiles
@@ -91,8 +84,8 @@ struct PairLayout {
   static constexpr int kKVFull = 2;                           // + stage
   static constexpr int kKVEmpty = kKVFull + kStages;          // + stage
   static constexpr int kSFull = kKVEmpty + kStages;           // + tile
-  static constexpr int kPFull = kSFull + 2;                   // + 2 * tile + half
-  static constexpr int kOUnit = kPFull + 4;                   // + tile: O of a unit complete
+  static constexpr int kPFull = kSFull + 2;                   // + tile
+  static constexpr int kOUnit = kPFull + 2;                   // + tile: O of a unit complete
   static constexpr int kOEmpty = kOUnit + 2;                  // + tile
   static constexpr int kStFull = kOEmpty + 2;                 // + tile
   static constexpr int kStEmpty = kStFull + 2;                // + tile
@@ -153,8 +146,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     for (int t = 0; t < 2; ++t) {
       ptx::mbar_init(bar(Lay::kSFull + t), 1);
-      ptx::mbar_init(bar(Lay::kPFull + 2 * t), 4);       // keys 0..63 of P: the tile's
-      ptx::mbar_init(bar(Lay::kPFull + 2 * t + 1), 4);   // softmax warps; the rest
+      ptx::mbar_init(bar(Lay::kPFull + t), 4);     // the tile's softmax warps
       ptx::mbar_init(bar(Lay::kOUnit + t), 1);
       ptx::mbar_init(bar(Lay::kOEmpty + t), 4);    // epilogue warps
       ptx::mbar_init(bar(Lay::kStFull + t), 4);
@@ -307,14 +299,6 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
               ptx::tmem_st_x16(t_s + ch * 16, pk);
             else
               ptx::tmem_st_x8(t_s + ch * 8, pk);
-            if (kPLoKeys > 0 && ch == kPLoKeys / (2 * kPk) - 1) {
-              // The first 64 keys' weights are in TMEM: their part of P_t V_j
-              // may start while the rest are formed.
-              ptx::tmem_wait_st();
-              ptx::tc_fence_before();
-              __syncwarp();
-              if (lane == 0) ptx::mbar_arrive(bar(Lay::kPFull + 2 * t));
-            }
           }
           float e0, e1;
           ptx::f2_unpack(ptx::f2_add(se[0], se[1]), e0, e1);
@@ -324,7 +308,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(Lay::kPFull + 2 * t + 1));
+        if (lane == 0) ptx::mbar_arrive(bar(Lay::kPFull + t));
       }
       if (!ok) break;
       if (!(ok = wait_warp(bar(Lay::kStEmpty + t), (st_cnt & 1) ^ 1, ctl))) break;
@@ -577,16 +561,14 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         if (commit) ptx::mma_commit(bar(Lay::kSFull + t));
       };
-      // O_t += P_t V with V in ring stage st: the products over keys
-      // [16 k0, 16 k1)
-      auto pv = [&](int t, int j, uint32_t st, int k0, int k1) {
+      // O_t += P_t V with V in ring stage st
+      auto pv = [&](int t, int j, uint32_t st) {
         const uint32_t b_lo = ring_lo + st * (Lay::kSlotBytes >> 4) + v_lbo;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          if (kk >= k0 && kk < k1)
-            ptx::mma_f16_ts(tmem + Lay::kTmemO + t * 128, tmem + t * 128 + kk * 8,
-                            ptx::sdesc_join(b_lo + kk * (2048 >> 4), kDescHi), kIdescO,
-                            (j == 0 && kk == 0) ? 0u : 1u);
+          ptx::mma_f16_ts(tmem + Lay::kTmemO + t * 128, tmem + t * 128 + kk * 8,
+                          ptx::sdesc_join(b_lo + kk * (2048 >> 4), kDescHi), kIdescO,
+                          (j == 0 && kk == 0) ? 0u : 1u);
       };
       for (uint32_t k = 0; ok; ++k) {
         const uint32_t uslot = k % kUnitSlots;
@@ -616,16 +598,10 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           bool k_taken = false;
           for (int t = 0; t < 2; ++t) {
             if (j >= n_t[t]) continue;
-            if (!(ok = wait_one(bar(Lay::kPFull + 2 * t + (kPLoKeys > 0 ? 0 : 1)), g[t] & 1, ctl)))
-              break;
+            if (!(ok = wait_one(bar(Lay::kPFull + t), g[t] & 1, ctl))) break;
             if (j == 0 && !(ok = wait_one(bar(Lay::kOEmpty + t), (oe_cnt[t] & 1) ^ 1, ctl))) break;
             ptx::tc_fence_after();
-            if (kPLoKeys > 0) {
-              pv(t, j, st_v, 0, kPLoKeys / 16);
-              if (!(ok = wait_one(bar(Lay::kPFull + 2 * t + 1), g[t] & 1, ctl))) break;
-              ptx::tc_fence_after();
-            }
-            pv(t, j, st_v, kPLoKeys / 16, BN / 16);
+            pv(t, j, st_v);
             if (j == n_t[t] - 1) {
               ptx::mma_commit(bar(Lay::kOUnit + t));
               ++oe_cnt[t];
