@@ -234,42 +234,11 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           for (int q = 0; q < BN; ++q)
             if (q >= limit) s[q] = -INFINITY;
         }
-        float mx[8];
-#pragma unroll
-        for (int a = 0; a < 8; ++a) mx[a] = fmaxf(s[2 * a], s[2 * a + 1]);
-#pragma unroll
-        for (int q = 16; q < BN; q += 16)
-#pragma unroll
-          for (int a = 0; a < 8; ++a) mx[a] = ptx::fmax3(mx[a], s[q + 2 * a], s[q + 2 * a + 1]);
-        const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
-        if (j == 0) {
-          m_used = m_tile;
-        } else {
-          // Rescale only rows whose maximum grew past the threshold (warp-wide
-          // TMEM access: other rows take part with a factor of exactly 1).
-          // S_t(j) completed after P_t V_{j-1}, so O_t is up to date.
-          const bool need = m_tile > m_used + kRescaleTau;
-          if (__any_sync(0xffffffffu, need)) {
-            const float m_next = need ? m_tile : m_used;
-            const float alpha = need ? ptx::ex2_approx(m_used - m_next) : 1.f;
-#pragma unroll
-            for (int cc = 0; cc < D / 16; ++cc) {
-              uint32_t o[16];
-              ptx::tmem_ld_x16(t_o + cc * 16, o);
-#pragma unroll
-              for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-              ptx::tmem_st_x16(t_o + cc * 16, o);
-            }
-            l *= alpha;
-            l_round *= alpha;
-            m_used = m_next;
-          }
-        }
-        // Weights rounded to bf16 for the P V product; O is divided by the
-        // sum of the rounded weights, the log-sum-exp uses the exact sum.
-        {
-          const float base = m_used == -INFINITY ? 0.f : m_used;
+        // Weights rounded to bf16 for the P V product, written over the
+        // scores; returns the sums of the weights (for the log-sum-exp) and
+        // of the rounded weights (O is divided by the latter).
+        auto weights = [&](float base_in, float& e_sum, float& r_sum) {
+          const float base = base_in == -INFINITY ? 0.f : base_in;
           const uint64_t nb2 = ptx::f2_pack(-base, -base);
           uint64_t se[2];
           float sr[4];
@@ -302,9 +271,51 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           }
           float e0, e1;
           ptx::f2_unpack(ptx::f2_add(se[0], se[1]), e0, e1);
-          l += e0 + e1;
-          l_round += (sr[0] + sr[1]) + (sr[2] + sr[3]);
+          e_sum = e0 + e1;
+          r_sum = (sr[0] + sr[1]) + (sr[2] + sr[3]);
+        };
+        // Lazy rescale: rows whose maximum grew past the threshold take the
+        // new maximum and O_t's rows are multiplied by 2^(m_old - m_new)
+        // (warp-wide TMEM access: other rows take part with a factor of
+        // exactly 1).  S_t(j) completed after P_t V_{j-1}, so O_t is up to
+        // date.
+        auto rescale = [&](bool need, float m_tile) {
+          const float m_next = need ? m_tile : m_used;
+          const float alpha = need ? ptx::ex2_approx(m_used - m_next) : 1.f;
+#pragma unroll
+          for (int cc = 0; cc < D / 16; ++cc) {
+            uint32_t o[16];
+            ptx::tmem_ld_x16(t_o + cc * 16, o);
+#pragma unroll
+            for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+            ptx::tmem_st_x16(t_o + cc * 16, o);
+          }
+          l *= alpha;
+          l_round *= alpha;
+          m_used = m_next;
+        };
+        auto tile_max = [&]() -> float {
+          float mx[8];
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx[a] = fmaxf(s[2 * a], s[2 * a + 1]);
+#pragma unroll
+          for (int q = 16; q < BN; q += 16)
+#pragma unroll
+            for (int a = 0; a < 8; ++a) mx[a] = ptx::fmax3(mx[a], s[q + 2 * a], s[q + 2 * a + 1]);
+          return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
+        };
+        const float m_tile = tile_max();
+        if (j == 0) {
+          m_used = m_tile;
+        } else {
+          const bool need = m_tile > m_used + kRescaleTau;
+          if (__any_sync(0xffffffffu, need)) rescale(need, m_tile);
         }
+        float e_sum, r_sum;
+        weights(m_used, e_sum, r_sum);
+        l += e_sum;
+        l_round += r_sum;
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
