@@ -261,9 +261,9 @@ EXTRA_WORKLOADS = ("packed_causal", "long_outlier", "mxfp8_packed", "mxfp8_incoh
 
 
 def kernel_name_for(dtype_name: str) -> str:
-    """bf16 runs the two-query-tile kernel, MXFP8 and NVFP4 (head dim 128)
-    the block-scaled one."""
-    return "attn_fwd_kernel" if dtype_name in ("mxfp8", "nvfp4") else "attn_fwd_pair_kernel"
+    """Every forward form (bf16, MXFP8, NVFP4) runs the two-query-tile
+    kernel."""
+    return "attn_fwd_pair_kernel"
 
 
 def measure_workload(A, name, steps, warmup, dev, stream, pg, clk):

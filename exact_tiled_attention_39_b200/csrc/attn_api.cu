@@ -52,12 +52,6 @@ void timing_mark(int i, cudaStream_t strm) {
   if (cudaEventRecord(g_timing.ev[i], strm) == cudaSuccess && i == 2) g_timing.recorded = true;
 }
 
-// MXFP8 at head dim 128 on the two-query-tile kernel (else the one-tile one).
-#ifndef ATTN_MXFP8_PAIR
-#define ATTN_MXFP8_PAIR 1
-#endif
-constexpr bool kMxfp8Pair = ATTN_MXFP8_PAIR != 0;
-
 constexpr int kMaxDevices = 64;
 constexpr int kScheduleThreads = 1024;
 constexpr int kSortCapacityMax = 16384;                   // 128 KB of keys
@@ -152,12 +146,9 @@ attn_status_t device_info(int* dev_out, DeviceInfo* info) {
   if (!d.ready) {
     if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    if (cudaFuncSetAttribute(attn_fwd_kernel<128, kQkMx8>,
+    if (cudaFuncSetAttribute(attn_fwd_pair_kernel<128, kQkNv4>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FwdLayout<128, kQkMx8>::kBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(attn_fwd_kernel<128, kQkNv4>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             FwdLayout<128, kQkNv4>::kBytes) != cudaSuccess ||
+                             PairLayout<128, kQkNv4>::kBytes) != cudaSuccess ||
         cudaFuncSetAttribute(attn_fwd_pair_kernel<64, kQkBf16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              PairLayout<64, kQkBf16>::kBytes) != cudaSuccess ||
@@ -197,13 +188,15 @@ bool encode_qkv_map(CUtensorMap* m, const void* base, int T, int H, int d, int e
 }
 
 // 3-D map over packed E2M1 codes [T, H, d / 2 bytes]: box = the d / 2 bytes
-// of a row (64 for d = 128) x 1 head x 128 tokens, 64-byte swizzle.
-bool encode_fp4_map(CUtensorMap* m, const void* base, int T, int H, int d) {
+// of a row (64 for d = 128) x 1 head x box_rows tokens, 64-byte swizzle.
+bool encode_fp4_map(CUtensorMap* m, const void* base, int T, int H, int d,
+                    int box_rows = kBlockM) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d / 2), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(T)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d / 2),
                                  static_cast<cuuint64_t>(H) * (d / 2)};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(d / 2), 1, static_cast<cuuint32_t>(kBlockM)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(d / 2), 1,
+                             static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[3] = {1, 1, 1};
   return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -292,19 +285,17 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* header = reinterpret_cast<int32_t*>(ws);
 
-  // bf16 and MXFP8 (d = 128) run the two-query-tile kernel (MXFP8 with
-  // 112-key tiles), NVFP4 (d = 128) the one-tile block-scaled kernel.
+  // Every path runs the two-query-tile kernel; the block-scaled forms
+  // (MXFP8, NVFP4 at d = 128) with 112-key tiles.
   const bool nv4 = dtype == ATTN_NVFP4;
   const bool fp8_kernel = (dtype == ATTN_MXFP8 || nv4) && s.head_dim == 128;
-  const bool mx8_pair = fp8_kernel && !nv4 && kMxfp8Pair;
-  const bool pair_kernel = !fp8_kernel || mx8_pair;
-  const int kv_rows = mx8_pair ? PairLayout<128, kQkMx8>::kBN : kBlockN;
+  const int kv_rows = fp8_kernel ? PairLayout<128, kQkMx8>::kBN : kBlockN;
   timing_mark(0, strm);
   // 1. schedule (validates cu_seqlens, writes the work list and its length)
   const int64_t cap = sort_capacity_for(wl.max_entries);
   build_schedule_kernel<<<1, kScheduleThreads, static_cast<size_t>(cap) * 8, strm>>>(
       cu_seqlens, s.num_seqs, s.total_tokens, s.max_seqlen, s.max_seqlen, causal,
-      pair_kernel ? 2 : 1, header,
+      2, header,
       reinterpret_cast<int4*>(ws + wl.sorted_off), reinterpret_cast<int4*>(ws + wl.unsorted_off),
       static_cast<int>(cap));
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -394,7 +385,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
   CUtensorMap tq, tk, tv;
   if (fp8_kernel && nv4) {
     if (!encode_fp4_map(&tq, qk_src[0], s.total_tokens, s.num_heads, s.head_dim) ||
-        !encode_fp4_map(&tk, qk_src[1], s.total_tokens, s.num_heads, s.head_dim))
+        !encode_fp4_map(&tk, qk_src[1], s.total_tokens, s.num_heads, s.head_dim, kv_rows))
       return ATTN_ERR_CUDA;
   } else if (!encode_qkv_map(&tq, qk_src[0], s.total_tokens, s.num_heads, s.head_dim, qk_elem) ||
              !encode_qkv_map(&tk, qk_src[1], s.total_tokens, s.num_heads, s.head_dim, qk_elem,
@@ -427,21 +418,18 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(pair_kernel ? kPairThreads : kFwdThreads);
+  cfg.blockDim = dim3(kPairThreads);
   cfg.stream = strm;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
   timing_mark(1, strm);
   if (fp8_kernel && nv4) {
-    cfg.dynamicSmemBytes = FwdLayout<128, kQkNv4>::kBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, kQkNv4>, tq, tk, tv, fp);
-  } else if (mx8_pair) {
+    cfg.dynamicSmemBytes = PairLayout<128, kQkNv4>::kBytes;
+    e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<128, kQkNv4>, tq, tk, tv, fp);
+  } else if (fp8_kernel) {
     cfg.dynamicSmemBytes = PairLayout<128, kQkMx8>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<128, kQkMx8>, tq, tk, tv, fp);
-  } else if (fp8_kernel) {
-    cfg.dynamicSmemBytes = FwdLayout<128, kQkMx8>::kBytes;
-    e = cudaLaunchKernelEx(&cfg, attn_fwd_kernel<128, kQkMx8>, tq, tk, tv, fp);
   } else if (s.head_dim == 128) {
     cfg.dynamicSmemBytes = PairLayout<128, kQkBf16>::kBytes;
     e = cudaLaunchKernelEx(&cfg, attn_fwd_pair_kernel<128, kQkBf16>, tq, tk, tv, fp);

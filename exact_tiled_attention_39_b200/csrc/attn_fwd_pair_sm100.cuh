@@ -1,5 +1,7 @@
-// Exact attention forward for sm_100a, bf16: two query tiles per CTA sharing
-// every K/V tile, one softmax warpgroup per query tile.
+// Exact attention forward for sm_100a: two query tiles per CTA sharing every
+// K/V tile, one softmax warpgroup per query tile.  The score product runs in
+// bf16, or block-scaled on MXFP8 or NVFP4 codes (head dim 128, 112-key
+// tiles); P V always runs in bf16.
 //
 // The method is the one of attn_fwd_sm100.cuh ("FlashAttention và IO"
 // (aihero.vn), sections "Tiling giữ công việc ở gần nơi tính" and "Softmax
@@ -23,8 +25,10 @@
 //   warps 4..7    softmax of tile B.
 //   warps 8..11   epilogue (64 registers): O_t / l_round -> bf16, lse.
 //   warp 12       producer (80 registers): claims units, TMA loads of Q_A,
-//                 Q_B and of K_j, V_j into a ring of shared-memory slots.
-//   warp 13       MMA issuer (one thread).
+//                 Q_B and of K_j, V_j into a ring of shared-memory slots;
+//                 block-scaled forms: the whole warp stages the scale blocks.
+//   warp 13       MMA issuer (one thread); block-scaled forms: copies the
+//                 scale blocks into TMEM (tcgen05.cp) ahead of the products.
 //   warps 14..15  idle.
 //
 // TMEM (512 columns, lane = query row): S_A at 0, S_B at 128, O_A at 256,
@@ -50,25 +54,30 @@ static_assert(2 * kPairRegsSoftmax + kPairRegsEpilogue + kPairRegsOther == 4 * 1
               "register split must use exactly the registers the CTA is launched with");
 constexpr int kPairUnitConsumers = 1 + 8 + 4;   // MMA thread + softmax warps + epilogue warps
 
-// Score operand format kQk (attn_fwd_sm100.cuh): bf16, or MXFP8 (E4M3 codes
-// with one E8M0 scale per 32 elements; head dim 128).  MXFP8 uses key tiles
-// of 112: the score products are then 112 columns wide, which leaves the
-// last 16 columns of each tile's score buffer for the scale factors (Q's
-// of each tile, and two buffers of the K tile's).
+// Score operand format kQk (attn_fwd_sm100.cuh): bf16; MXFP8 (E4M3 codes
+// with one E8M0 scale per 32 elements); NVFP4 (packed E2M1 codes with one
+// UE4M3 scale per 16 elements); the block-scaled formats at head dim 128.
+// They use key tiles of 112: the score products are then 112 columns wide,
+// which leaves the last 16 columns of each tile's score buffer for the
+// scale factors (Q's of each tile, and two buffers of the K tile's).
 template <int D, int kQk>
 struct PairLayout {
-  static constexpr bool kFp8 = kQk == kQkMx8;
-  static_assert(kQk == kQkBf16 || kQk == kQkMx8, "pair kernel: bf16 or MXFP8 score operands");
+  static constexpr bool kFp8 = kQk != kQkBf16;                // block-scaled Q, K
+  static constexpr bool kNv4 = kQk == kQkNv4;
   static_assert(D == 64 || D == 128, "head dim 64 or 128");
-  static_assert(!kFp8 || D == 128, "MXFP8 pair kernel: head dim 128");
+  static_assert(!kFp8 || D == 128, "block-scaled pair kernel: head dim 128");
   static constexpr int kBN = kFp8 ? 112 : 128;                // keys per K/V tile
   static constexpr int kChunks = D / 64;                      // 128-byte chunks of a bf16 row
-  static constexpr int kQkChunks = kFp8 ? 1 : kChunks;        // ... of a Q or K row
-  static constexpr int kQTileBytes = kQkChunks * kBlockM * 128;
-  static constexpr int kKTileBytes = kQkChunks * kBN * 128;
+  static constexpr int kQkChunks = kFp8 ? 1 : kChunks;        // swizzle chunks of a Q or K row
+  static constexpr int kQkRowBytes = kNv4 ? 64 : 128;         // bytes of a Q or K row per chunk
+  static constexpr int kQTileBytes = kQkChunks * kBlockM * kQkRowBytes;
+  static constexpr int kKTileBytes = kQkChunks * kBN * kQkRowBytes;
   static constexpr int kVChunkBytes = kBN * 128;
   static constexpr int kVTileBytes = kChunks * kVChunkBytes;
-  static constexpr int kSfBytes = kFp8 ? 512 : 0;             // scale block of a Q or K tile
+  // Scale words per row (4 scale bytes each): MXFP8 1, NVFP4 2 (one per
+  // K = 64 product); one 32-row x 16-byte block per word and tile.
+  static constexpr int kSfWords = kNv4 ? 2 : 1;
+  static constexpr int kSfBytes = kFp8 ? 512 * kSfWords : 0;  // scale blocks of a Q or K tile
   static constexpr int kSlotRaw = kVTileBytes > kKTileBytes + kSfBytes ? kVTileBytes
                                                                        : kKTileBytes + kSfBytes;
   static constexpr int kSlotBytes = (kSlotRaw + 1023) / 1024 * 1024;   // a K (+ scales) or V tile
@@ -102,9 +111,13 @@ struct PairLayout {
   static_assert(kSlotBytes % 1024 == 0 && kVChunkBytes % 1024 == 0, "swizzle alignment");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemO = 256;                     // + 128 * tile
-  // MXFP8 scale factors in the unused columns 112..127 of the score buffers:
-  // Q_t's at 128 t + 112, the K tiles' (two buffers) at 116 and 120.
-  static constexpr uint32_t kTmemSfa = 112, kTmemSfb = 116;
+  // Scale factors in the unused columns 112..127 of the score buffers, 4
+  // columns per scale word: Q_t's at 128 t + 112; the K tiles' two buffers
+  // at 116 and 120 (MXFP8) or 120 and 248 (NVFP4, 8 columns each).
+  static constexpr uint32_t kTmemSfa = 112;
+  __host__ __device__ static constexpr uint32_t sfb_col(uint32_t b) {
+    return kNv4 ? 120 + 128 * b : 116 + 4 * b;
+  }
 };
 
 // Key steps of query tile qb (128 rows) of a document of doc_len tokens with
@@ -392,14 +405,16 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       // Scale block of the 128 rows from row0 (MXFP8): lane m0 writes rows
       // m0 + 32 c, c = 0..3, as 16 bytes at offset 16 m0 (the layout
       // tcgen05.cp replicates); rows past `rows` or the tensor get 0.
-      auto stage_scales = [&](const uint32_t* scales, int head, int row0, int rows, int off) {
+      auto stage_scales = [&](const uint32_t* scales, int head, int row0, int rows, int w,
+                              int off) {
         uint32_t wv[4];
 #pragma unroll
         for (int cq = 0; cq < 4; ++cq) {
           const int rr = lane + 32 * cq;
           const int tok = row0 + rr;
           wv[cq] = rr < rows && tok < p.total_tokens
-                       ? scales[static_cast<long long>(tok) * H + head] : 0u;
+                       ? scales[(static_cast<long long>(tok) * H + head) * Lay::kSfWords + w]
+                       : 0u;
         }
         *reinterpret_cast<uint4*>(smem + off + 16 * lane) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
       };
@@ -408,8 +423,9 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const uint32_t s = kv_it % Lay::kStages;
         if (!wait_warp(bar(Lay::kKVEmpty + s), ((kv_it / Lay::kStages) & 1) ^ 1, ctl)) return false;
         if (kFp8 && kind == 0) {
-          stage_scales(p.k_scales, head, row0, BN,
-                       Lay::kRingOff + s * Lay::kSlotBytes + Lay::kKTileBytes);
+          for (int w = 0; w < Lay::kSfWords; ++w)
+            stage_scales(p.k_scales, head, row0, BN, w,
+                         Lay::kRingOff + s * Lay::kSlotBytes + Lay::kKTileBytes + 512 * w);
           fence_proxy_async_smem();
           __syncwarp();
         }
@@ -419,7 +435,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             ptx::mbar_arrive_expect_tx(bar(Lay::kKVFull + s), Lay::kKTileBytes);
             for (int cq = 0; cq < Lay::kQkChunks; ++cq)
               ptx::tma_load_3d(slot + cq * BN * 128, &tm_k, bar(Lay::kKVFull + s),
-                               cq * (kFp8 ? 128 : 64), head, row0);
+                               cq * 64, head, row0);
           } else {
             ptx::mbar_arrive_expect_tx(bar(Lay::kKVFull + s), Lay::kVTileBytes);
             for (int cq = 0; cq < Lay::kChunks; ++cq)
@@ -475,8 +491,9 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const int qrow0 = uw.x + 2 * kBlockM * uw.z;
         if constexpr (kFp8) {
           for (int t = 0; t < 2; ++t)
-            stage_scales(p.q_scales, uw.w, qrow0 + t * kBlockM, kBlockM,
-                         Lay::kSfaOff + t * Lay::kSfBytes);
+            for (int w = 0; w < Lay::kSfWords; ++w)
+              stage_scales(p.q_scales, uw.w, qrow0 + t * kBlockM, kBlockM, w,
+                           Lay::kSfaOff + t * Lay::kSfBytes + 512 * w);
           fence_proxy_async_smem();
           __syncwarp();
         }
@@ -485,8 +502,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           for (int t = 0; t < 2; ++t)
             for (int cq = 0; cq < Lay::kQkChunks; ++cq)
               ptx::tma_load_3d(sbase + Lay::kQOff + t * Lay::kQTileBytes + cq * kBlockM * 128,
-                               &tm_q, bar(Lay::kQFull), cq * (kFp8 ? 128 : 64), uw.w,
-                               qrow0 + t * kBlockM);
+                               &tm_q, bar(Lay::kQFull), cq * 64, uw.w, qrow0 + t * kBlockM);
         }
         __syncwarp();
         ++q_it;
@@ -512,6 +528,8 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       constexpr uint32_t kIdescS = ptx::idesc_bf16(kBlockM, BN, 0);
       constexpr uint32_t kIdescO = ptx::idesc_bf16(kBlockM, D, 1);
       constexpr uint32_t kDescHi = ptx::sdesc_hi_sw128(1024);
+      // NVFP4 Q and K rows are 64 bytes: 64-byte swizzle, 8-row groups 512 B apart
+      constexpr uint32_t kQkDescHi = Lay::kNv4 ? ptx::sdesc_hi_sw64(512) : kDescHi;
       const uint32_t q_lo = ptx::sdesc_lo(sbase + Lay::kQOff, 16);
       const uint32_t ring_lo = ptx::sdesc_lo(sbase + Lay::kRingOff, 16);
       const uint32_t v_lbo = static_cast<uint32_t>(Lay::kVChunkBytes - 16) >> 4 << 16;
@@ -530,16 +548,18 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         return r2;
       };
-      // The next K tile; MXFP8: its scale block into the next TMEM buffer
-      // (the products that read that buffer two K tiles ago were issued
-      // before, and the tensor pipe keeps issue order).
+      // The next K tile; block-scaled: its scale blocks into the next TMEM
+      // buffer (the products that read that buffer two K tiles ago were
+      // issued before, and the tensor pipe keeps issue order).
       auto take_k = [&](uint32_t& st) -> bool {
         if (!take(st)) return false;
         if constexpr (kFp8) {
           ptx::tc_fence_after();
-          tmem_cp_32x128b_x4(tmem + Lay::kTmemSfb + 4 * (k_cnt & 1),
-                             sf_copy_desc(sbase + Lay::kRingOff + st * Lay::kSlotBytes +
-                                          Lay::kKTileBytes));
+#pragma unroll
+          for (int w = 0; w < Lay::kSfWords; ++w)
+            tmem_cp_32x128b_x4(tmem + Lay::sfb_col(k_cnt & 1) + 4 * w,
+                               sf_copy_desc(sbase + Lay::kRingOff + st * Lay::kSlotBytes +
+                                            Lay::kKTileBytes + 512 * w));
         }
         ++k_cnt;
         return true;
@@ -548,11 +568,23 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       auto score = [&](int t, uint32_t st, bool commit = true) {
         const uint32_t a_lo = q_lo + ((t * Lay::kQTileBytes) >> 4);
         const uint32_t b_lo = ring_lo + st * (Lay::kSlotBytes >> 4);
-        if constexpr (kFp8) {
+        if constexpr (Lay::kNv4) {
+          // block-scaled E2M1: two K = 64 products (32 bytes of packed codes
+          // each, 64-byte swizzle), scale word kk of each row
+          const uint32_t sfa = tmem + t * 128 + Lay::kTmemSfa;
+          const uint32_t sfb = tmem + Lay::sfb_col((k_cnt - 1) & 1);
+#pragma unroll
+          for (int kk = 0; kk < D / 64; ++kk) {
+            const uint32_t off = (kk * 32) >> 4;
+            mma_nvf4_ss(tmem + t * 128, ptx::sdesc_join(a_lo + off, kQkDescHi),
+                        ptx::sdesc_join(b_lo + off, kQkDescHi), idesc_nvf4(BN), sfa + 4 * kk,
+                        sfb + 4 * kk, kk > 0 ? 1u : 0u);
+          }
+        } else if constexpr (kFp8) {
           // block-scaled E4M3: four K = 32 products, scale byte kk of each
           // row's word
           const uint32_t sfa = tmem + t * 128 + Lay::kTmemSfa;
-          const uint32_t sfb = tmem + Lay::kTmemSfb + 4 * ((k_cnt - 1) & 1);
+          const uint32_t sfb = tmem + Lay::sfb_col((k_cnt - 1) & 1);
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk) {
             const uint32_t off = (kk * 32) >> 4;
@@ -595,8 +627,9 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::tc_fence_after();
         if constexpr (kFp8) {
           for (int t = 0; t < 2; ++t)
-            tmem_cp_32x128b_x4(tmem + t * 128 + Lay::kTmemSfa,
-                               sf_copy_desc(sbase + Lay::kSfaOff + t * Lay::kSfBytes));
+            for (int w = 0; w < Lay::kSfWords; ++w)
+              tmem_cp_32x128b_x4(tmem + t * 128 + Lay::kTmemSfa + 4 * w,
+                                 sf_copy_desc(sbase + Lay::kSfaOff + t * Lay::kSfBytes + 512 * w));
         }
         uint32_t st_k, st_v;
         if (!(ok = take_k(st_k))) break;
