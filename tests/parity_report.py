@@ -1,4 +1,5 @@
-"""Parity figures of the five configurations, one JSON line each (GPU).
+"""Parity figures of the five configurations, the NVFP4 / FP8 mixed path and
+incoherent processing, one JSON line each (GPU).
 
     python tests/parity_report.py [--bwd-only]
 
@@ -124,6 +125,29 @@ def main():
         le = np.abs(lse.double().numpy() - rl)
         out_lines.append(line(name, ro.shape[0] * ro.shape[1], e, le,
                               MXFP8_MAX_ABS if fp8 else BF16_MAX_ABS, BF16_MEAN_ABS))
+    # NVFP4 Q, K with MXFP8 V, against the oracle on the exactly dequantised inputs
+    from oracle.nvfp4 import dequantize_nvfp4_ref, quantize_nvfp4_ref
+    inp = workloads.make_inputs("nvfp4_packed")
+    out, lse, _ = run_gpu(inp["q"], inp["k"], inp["v"], inp["cu_seqlens"], True, inp["scale"],
+                          dtype=A.ATTN_NVFP4, max_seqlen=max(inp["lengths"]))
+    qd = dequantize_nvfp4_ref(*quantize_nvfp4_ref(inp["q"].double().numpy()))
+    kd = dequantize_nvfp4_ref(*quantize_nvfp4_ref(inp["k"].double().numpy()))
+    ro, rl = full_reference(qd, kd, deq(inp["v"]), inp["lengths"], True, inp["scale"])
+    out_lines.append(line("nvfp4_packed", ro.shape[0] * ro.shape[1],
+                          np.abs(out.double().numpy() - ro), np.abs(lse.double().numpy() - rl),
+                          MXFP8_MAX_ABS, BF16_MEAN_ABS))
+    # incoherent processing, against the oracle of the rotated, quantised operands
+    from oracle.incoherent import incoherent_operands
+    from test_gpu_incoherent import _run_incoherent
+    inp = workloads.make_inputs("mxfp8_incoherent")
+    out, lse = _run_incoherent(inp["q"], inp["k"], inp["v"], inp["cu_seqlens"], True,
+                               inp["scale"], inp["signs"], max(inp["lengths"]))
+    q, k, v = (inp[n].double().numpy() for n in ("q", "k", "v"))
+    qd, kd, vd, s = incoherent_operands(q, k, v, inp["scale"], inp["signs"].numpy())
+    ro, rl = full_reference(qd, kd, vd, inp["lengths"], True, s)
+    out_lines.append(line("mxfp8_incoherent", ro.shape[0] * ro.shape[1],
+                          np.abs(out.double().numpy() - ro), np.abs(lse.double().numpy() - rl),
+                          MXFP8_MAX_ABS, BF16_MEAN_ABS))
     out_lines += bwd_lines()
     for l_ in out_lines:
         print(json.dumps(l_))
