@@ -320,8 +320,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
       jobs.t[i].deq = use_codes ? nullptr : reinterpret_cast<uint4*>(ws + wl.deq_off[i]);
       jobs.t[i].rotate = i < 2 ? 1 : 0;
     }
-    // D / 8 lanes per row, 256 threads per block
-    const long long rows_per_block = 256 / (s.head_dim / 8);
+    // D / 8 lanes per row, 256 threads per block, kRotRowsPerThread rows a thread
+    const long long rows_per_block = 256 / (s.head_dim / 8) * kRotRowsPerThread;
     const long long qgrid = (jobs.rows + rows_per_block - 1) / rows_per_block;
     if (qgrid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     if (s.head_dim == 128)
@@ -350,7 +350,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, const int32_
       jobs.scales[i] = fp8_kernel ? ws + wl.scales_off[i] : nullptr;
     }
     jobs.n16 = static_cast<long long>(s.total_tokens) * s.num_heads * (s.head_dim / 16);
-    const long long qgrid = (jobs.n16 + 255) / 256;
+    const long long qgrid = (jobs.n16 / 2 + 255) / 256;     // one thread per 32 elements
     if (qgrid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
     quantize_nvfp4_qk_mxfp8_v_kernel<<<dim3(static_cast<unsigned>(qgrid), 3), 256, 0, strm>>>(jobs);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -772,7 +772,7 @@ extern "C" attn_status_t attn_quantize_mxfp8_rotated(const void* x, const float*
     return ATTN_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u) != 0)
     return ATTN_ERR_ALIGNMENT;
-  const long long rows_per_block = 256 / (cols / 8);
+  const long long rows_per_block = 256 / (cols / 8) * kRotRowsPerThread;
   const long long grid = (rows + rows_per_block - 1) / rows_per_block;
   if (grid > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   cudaStream_t strm = static_cast<cudaStream_t>(stream);

@@ -45,29 +45,26 @@ struct RowQuantJobs {
 // element of a pair becomes a + b, the upper a - b, the same fp32 additions
 // in the same order as one thread per row would make.  A 32-element
 // quantisation block is four lanes; its maximum comes from two shuffles.
-// Every lane of the warp must call this (rows past the end pass valid = 0).
+// Every lane of the warp must call this (rows past the end pass valid = 0);
+// w is the lane's 16 bytes of the row (loaded by the caller, so that several
+// rows' loads are in flight at once), sg the lane's 8 signs.
 template <int D>
-__device__ __forceinline__ void quantize_row_lanes(const RowQuantJob& j,
-                                                   const float* __restrict__ signs,
-                                                   long long row, bool valid) {
+__device__ __forceinline__ void quantize_row_lanes(const RowQuantJob& j, const float (&sg)[8],
+                                                   long long row, bool valid, uint4 w) {
   constexpr int kLanes = D / 8;
   const int sub = static_cast<int>(threadIdx.x) & (kLanes - 1);
   float y[8];
-  if (valid) {
-    const uint4 w = j.x[row * kLanes + sub];
+  {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       y[2 * q] = bf16_lo(ws[q]);
       y[2 * q + 1] = bf16_hi(ws[q]);
     }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] = 0.f;
   }
   if (j.rotate) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] *= signs[8 * sub + e];          // exact: +-1
+    for (int e = 0; e < 8; ++e) y[e] *= sg[e];                      // exact: +-1
 #pragma unroll
     for (int h = 1; h < 8; h <<= 1) {
 #pragma unroll
@@ -124,6 +121,37 @@ __device__ __forceinline__ void quantize_row_lanes(const RowQuantJob& j,
   }
 }
 
+// Rows per thread of the rotating kernels: a 256-thread block takes
+// kRotRowsPerThread groups of 256 / (D / 8) consecutive rows, and each
+// thread loads its rows' 16 bytes before working on the first, so that
+// several loads per thread are in flight (one is too few to keep HBM busy).
+constexpr int kRotRowsPerThread = 4;
+
+template <int D>
+__device__ __forceinline__ void quantize_rows_block(const RowQuantJob& j,
+                                                    const float* __restrict__ signs,
+                                                    long long rows) {
+  constexpr int kLanes = D / 8;
+  constexpr int kRowsPerPass = 256 / kLanes;
+  const int sub = static_cast<int>(threadIdx.x) & (kLanes - 1);
+  const long long row0 = static_cast<long long>(blockIdx.x) * (kRowsPerPass * kRotRowsPerThread) +
+                         static_cast<int>(threadIdx.x) / kLanes;
+  float sg[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) sg[e] = j.rotate ? signs[8 * sub + e] : 1.f;
+  uint4 w[kRotRowsPerThread];
+#pragma unroll
+  for (int i = 0; i < kRotRowsPerThread; ++i) {
+    const long long row = row0 + i * kRowsPerPass;
+    w[i] = row < rows ? j.x[row * kLanes + sub] : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int i = 0; i < kRotRowsPerThread; ++i) {
+    const long long row = row0 + i * kRowsPerPass;
+    quantize_row_lanes<D>(j, sg, row, row < rows, w[i]);
+  }
+}
+
 // Rows of D bf16 values, D / 8 lanes each: codes [rows][D] (E4M3), scales
 // [rows][D / 32] (E8M0), signs: D fp32 values (+-1).
 template <int D>
@@ -132,9 +160,8 @@ quantize_mxfp8_rotated_kernel(const uint4* __restrict__ x, const float* __restri
                               uint2* __restrict__ codes, uint8_t* __restrict__ scales,
                               long long rows) {
   static_assert(D == 64 || D == 128, "head dim 64 or 128");
-  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / (D / 8);
   const RowQuantJob j{x, codes, scales, nullptr, 1};
-  quantize_row_lanes<D>(j, signs, row, row < rows);
+  quantize_rows_block<D>(j, signs, rows);
 }
 
 // The pre-pass of an attention call with incoherent processing: Q and K
@@ -145,8 +172,7 @@ __global__ void __launch_bounds__(256)
 quantize_mxfp8_incoherent_qkv_kernel(const __grid_constant__ RowQuantJobs jobs,
                                      const float* __restrict__ signs) {
   static_assert(D == 64 || D == 128, "head dim 64 or 128");
-  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / (D / 8);
-  quantize_row_lanes<D>(jobs.t[blockIdx.y], signs, row, row < jobs.rows);
+  quantize_rows_block<D>(jobs.t[blockIdx.y], signs, jobs.rows);
 }
 
 }  // namespace attn

@@ -64,14 +64,13 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
   return (c & 8u) ? -mag : mag;
 }
 
-// One 16-element block b of a row-major bf16 tensor: codes (8 bytes),
-// scale byte and/or exact dequantised bf16 (32 bytes); any output may be
-// null.
-__device__ __forceinline__ void quantize_block_nvfp4(const uint4* __restrict__ x,
-                                                     uint2* __restrict__ codes,
-                                                     uint8_t* __restrict__ scales,
-                                                     uint4* __restrict__ deq, long long b) {
-  const uint4 v0 = x[2 * b], v1 = x[2 * b + 1];
+// One 16-element block b of a row-major bf16 tensor, given as its two
+// 16-byte halves v0, v1: codes (8 bytes), scale byte and/or exact
+// dequantised bf16 (32 bytes); any output may be null.
+__device__ __forceinline__ void quantize_block_nvfp4_values(uint4 v0, uint4 v1,
+                                                            uint2* __restrict__ codes,
+                                                            uint8_t* __restrict__ scales,
+                                                            uint4* __restrict__ deq, long long b) {
   const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
   float f[16];
   float amax = 0.f;
@@ -104,6 +103,13 @@ __device__ __forceinline__ void quantize_block_nvfp4(const uint4* __restrict__ x
   }
 }
 
+__device__ __forceinline__ void quantize_block_nvfp4(const uint4* __restrict__ x,
+                                                     uint2* __restrict__ codes,
+                                                     uint8_t* __restrict__ scales,
+                                                     uint4* __restrict__ deq, long long b) {
+  quantize_block_nvfp4_values(x[2 * b], x[2 * b + 1], codes, scales, deq, b);
+}
+
 // One thread per 16-element block; n_blocks = rows * cols / 16.
 __global__ void __launch_bounds__(256)
 quantize_nvfp4_kernel(const uint4* __restrict__ x, uint2* __restrict__ codes,
@@ -114,23 +120,29 @@ quantize_nvfp4_kernel(const uint4* __restrict__ x, uint2* __restrict__ codes,
 }
 
 // The pre-pass of the mixed path in one launch: blockIdx.y 0 and 1 take Q
-// and K to NVFP4 (one thread per 16-element block), 2 takes V to MXFP8
-// (one thread per 32-element block, exact dequantised bf16 only).
+// and K to NVFP4 (one thread per two consecutive 16-element blocks, both
+// loaded before either is worked on), 2 takes V to MXFP8 (one thread per
+// 32-element block, exact dequantised bf16 only): one thread per 32
+// elements and 64 bytes in flight in every part.
 struct MixedQuantJobs {
   const uint4* x[3];
   uint2* codes[2];        // packed E2M1 of Q, K (null: not written)
   uint8_t* scales[2];     // UE4M3 of Q, K (null: not written)
   uint4* deq[3];          // exact dequantised bf16 (null: not written)
-  long long n16;          // 16-element blocks per tensor
+  long long n16;          // 16-element blocks per tensor (even: rows of 64 or 128)
 };
 
 __global__ void __launch_bounds__(256)
 quantize_nvfp4_qk_mxfp8_v_kernel(const __grid_constant__ MixedQuantJobs jobs) {
   const long long b = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int t = blockIdx.y;
+  if (b >= jobs.n16 / 2) return;
   if (t < 2) {
-    if (b < jobs.n16) quantize_block_nvfp4(jobs.x[t], jobs.codes[t], jobs.scales[t], jobs.deq[t], b);
-  } else if (b < jobs.n16 / 2) {
+    const uint4* x = jobs.x[t];
+    const uint4 v0 = x[4 * b], v1 = x[4 * b + 1], v2 = x[4 * b + 2], v3 = x[4 * b + 3];
+    quantize_block_nvfp4_values(v0, v1, jobs.codes[t], jobs.scales[t], jobs.deq[t], 2 * b);
+    quantize_block_nvfp4_values(v2, v3, jobs.codes[t], jobs.scales[t], jobs.deq[t], 2 * b + 1);
+  } else {
     quantize_block(jobs.x[2], nullptr, nullptr, jobs.deq[2], b);
   }
 }
