@@ -39,9 +39,10 @@
 //                 bf16 values over the first 32 columns of its own 64, so
 //                 neither overwrites what the other has still to read.
 //   warps 8..11   dQ_i read-out (176 registers): TMEM -> registers -> shared
-//                 memory (the dS buffer, free once dQ_i's product has read
-//                 it) -> TMA reduce-add into the accumulator; at the end of a
-//                 unit the dK_j, dV_j epilogue.
+//                 memory (the ring stage of Q_i and dO_i, free once dK_i and
+//                 dV_i have read them; the producer refills it only after
+//                 these reductions have read it) -> TMA reduce-add into the
+//                 accumulator; at the end of a unit the dK_j, dV_j epilogue.
 //   warp 12       producer (80 registers): claims units; TMA loads of K_j,
 //                 V_j and of Q_i, dO_i into a two-stage ring, with the tile's
 //                 lse and D rows.
@@ -108,10 +109,11 @@ struct BwdLayout {
   static constexpr int kStageBytes = 2 * kTileBytes;          // Q_i, then dO_i
   static constexpr int kRingOff = 2 * kTileBytes;
   // dS (bf16, 128 queries x 128 keys), MN-major: row = key, 64 queries per
-  // 128-byte chunk row, two chunks of 16 KB.  Between dQ_i's product and
-  // the next dS it is the dQ staging area: per read-out warp two 4 KB
-  // buffers of 32 rows x 32 fp32 in the 128-byte swizzle.
+  // 128-byte chunk row, two chunks of 16 KB.
   static constexpr int kDsOff = kRingOff + kStages * kStageBytes;
+  // dQ_i staging, in ring stage i's Q_i (and, at head dim 64, dO_i) once
+  // dK_i and dV_i have read them: per read-out warp two 4 KB buffers of 32
+  // rows x 32 fp32 in the 128-byte swizzle.
   static constexpr int kStageBufBytes = 32 * 128;
   static constexpr int kDsBytes = 2 * kChunkBytes;
   static constexpr int kVecOff = kDsOff + kDsBytes;           // float [stage][lse2, D][128]
@@ -127,8 +129,7 @@ struct BwdLayout {
   static constexpr int kDQEmpty = kDQFull + 1;
   static constexpr int kDKVFull = kDQEmpty + 1;
   static constexpr int kDKVEmpty = kDKVFull + 1;
-  static constexpr int kDsFree = kDKVEmpty + 1;              // staging read by the reductions
-  static constexpr int kDrain = kDsFree + 1;
+  static constexpr int kDrain = kDKVEmpty + 1;
   static constexpr int kUnitFull = kDrain + 1;                // + slot
   static constexpr int kUnitEmpty = kUnitFull + kUnitSlots;   // + slot
   static constexpr int kNumBars = kUnitEmpty + kUnitSlots;
@@ -136,7 +137,7 @@ struct BwdLayout {
   static constexpr int kUnitOff = kMiscOff + 16;              // int4 [kUnitSlots]
   static constexpr int kBytes = kUnitOff + 16 * kUnitSlots;
   static_assert(kBytes <= 232448, "exceeds the 227 KB of shared memory per CTA");
-  static_assert(4 * 2 * kStageBufBytes <= kDsBytes, "dQ staging must fit the dS buffer");
+  static_assert(4 * 2 * kStageBufBytes <= kStageBytes, "dQ staging must fit a ring stage");
   static constexpr uint32_t kTmemS = 0;
   static constexpr uint32_t kTmemDP = 128;
   static constexpr uint32_t kTmemDV = 256;
@@ -239,7 +240,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     ptx::mbar_init(bar(Lay::kKVEmpty), 1);
     for (int s = 0; s < Lay::kStages; ++s) {
       ptx::mbar_init(bar(Lay::kQFull + s), 1);
-      ptx::mbar_init(bar(Lay::kQEmpty + s), 1 + kBwdComputeWarps);   // MMA + compute (lse, D)
+      // MMA (dK_i's product done) + compute warps (lse, D read) + read-out
+      // warps (dQ_i's staging read by its reductions)
+      ptx::mbar_init(bar(Lay::kQEmpty + s), 1 + kBwdComputeWarps + 4);
     }
     ptx::mbar_init(bar(Lay::kSFull), 1);
     ptx::mbar_init(bar(Lay::kPFull), kBwdComputeWarps);
@@ -249,7 +252,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     ptx::mbar_init(bar(Lay::kDQEmpty), 4);
     ptx::mbar_init(bar(Lay::kDKVFull), 1);
     ptx::mbar_init(bar(Lay::kDKVEmpty), 4);
-    ptx::mbar_init(bar(Lay::kDsFree), 4);
     ptx::mbar_init(bar(Lay::kDrain), 1);
     for (int i = 0; i < kUnitSlots; ++i) {
       ptx::mbar_init(bar(Lay::kUnitFull + i), 1);
@@ -359,8 +361,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // MN-major dS tile in shared memory
         if (!(ok = wait_warp(bar(Lay::kDPFull), q_cnt & 1, ctl))) break;
         ptx::tc_fence_after();
-        // the dS buffer: the previous step's dQ staging must have been read
-        if (q_cnt > 0 && !(ok = wait_warp(bar(Lay::kDsFree), (q_cnt - 1) & 1, ctl))) break;
+        // the dS buffer is free: dP^T of this step was issued after the
+        // previous dQ (the product that read dS) had left TMEM
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           uint32_t dp[32];
@@ -402,7 +404,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t stage_base = sbase + Lay::kDsOff + wq * 2 * Lay::kStageBufBytes;
+    const uint32_t warp_stage_off = wq * 2 * Lay::kStageBufBytes;
     uint32_t q_cnt = 0, u_cnt = 0;
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
@@ -437,7 +439,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
           }
-          const uint32_t buf = stage_base + (c & 1) * Lay::kStageBufBytes;
+          const uint32_t buf = sbase + Lay::kRingOff + (q_cnt % Lay::kStages) * Lay::kStageBytes +
+                               warp_stage_off + (c & 1) * Lay::kStageBufBytes;
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const uint32_t addr = buf + lane * 128 + ((u ^ (lane & 7)) << 4);
@@ -455,7 +458,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (lane == 0) bulk_wait_group_read<0>();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(Lay::kDsFree));
+        // the stage's staging has been read: the producer may refill it
+        if (lane == 0) ptx::mbar_arrive(bar(Lay::kQEmpty + q_cnt % Lay::kStages));
       }
       if (!ok) break;
       // dK_j, dV_j of the unit (key rows)
