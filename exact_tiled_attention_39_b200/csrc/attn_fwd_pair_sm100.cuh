@@ -329,6 +329,14 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         weights(m_used, e_sum, r_sum);
         l += e_sum;
         l_round += r_sum;
+        // bf16: a unit's first P goes to the tensor core only once the
+        // epilogue has read the previous unit's O_t (its first P V
+        // overwrites O_t), so the MMA thread's wait for P covers that and its
+        // issue loop carries no wait of its own (measured faster; the
+        // block-scaled forms keep the wait in the MMA thread, measured faster
+        // there).
+        if constexpr (!kFp8)
+          if (j == 0 && !(ok = wait_warp(bar(Lay::kOEmpty + t), (st_cnt & 1) ^ 1, ctl))) break;
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
@@ -535,7 +543,7 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const uint32_t v_lbo = static_cast<uint32_t>(Lay::kVChunkBytes - 16) >> 4 << 16;
       uint32_t q_ph = 0;
       uint32_t g[2] = {0, 0};          // key steps of each tile so far
-      uint32_t oe_cnt[2] = {0, 0};     // units of each tile so far
+      uint32_t oe_cnt[2] = {0, 0};     // units of each tile so far (block-scaled)
       uint32_t cur = 0, cur_ph = 0;    // ring cursor (stage, phase)
       uint32_t k_cnt = 0;              // K tiles taken (MXFP8: scale buffer k_cnt & 1)
       bool ok = true;
@@ -643,7 +651,9 @@ attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           for (int t = 0; t < 2; ++t) {
             if (j >= n_t[t]) continue;
             if (!(ok = wait_one(bar(Lay::kPFull + t), g[t] & 1, ctl))) break;
-            if (j == 0 && !(ok = wait_one(bar(Lay::kOEmpty + t), (oe_cnt[t] & 1) ^ 1, ctl))) break;
+            if constexpr (kFp8)
+              if (j == 0 && !(ok = wait_one(bar(Lay::kOEmpty + t), (oe_cnt[t] & 1) ^ 1, ctl)))
+                break;
             ptx::tc_fence_after();
             pv(t, j, st_v);
             if (j == n_t[t] - 1) {
