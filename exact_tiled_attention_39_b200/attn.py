@@ -264,13 +264,37 @@ def attn_bwd(q, k, v, out, dout, lse, cu_seqlens, dq, dk, dv, causal: bool, scal
     return workspace
 
 
+def _check_quant_args(x, codes, scales, code_bytes: int, scale_bytes: int, signs=None):
+    """Checks shared by the quantiser entry points; returns (rows, cols).
+    x: contiguous bf16 CUDA tensor whose last dimension is cols; codes and
+    scales: contiguous uint8 tensors on x's device holding exactly
+    code_bytes and scale_bytes per row (the library writes that many and
+    cannot see the buffers' sizes); signs, if given: fp32 [cols]."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() < 1:
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols > 0 else 0
+    for name, t, per_row in (("codes", codes, code_bytes), ("scales", scales, scale_bytes)):
+        if (t.dtype != torch.uint8 or not t.is_cuda or not t.is_contiguous()
+                or t.device != x.device or t.numel() != rows * per_row):
+            raise ValueError(f"{name} must be a contiguous uint8 tensor of {rows} x {per_row} "
+                             f"bytes on {x.device}")
+    if signs is not None and (signs.dtype != torch.float32 or not signs.is_cuda
+                              or not signs.is_contiguous() or tuple(signs.shape) != (cols,)
+                              or signs.device != x.device):
+        raise ValueError(f"signs must be a contiguous fp32 tensor of shape [{cols}] on {x.device}")
+    return rows, cols
+
+
 def attn_quantize_mxfp8(x, codes, scales, stream=None):
     """E4M3 + E8M0 quantisation of a bf16 [rows, cols] CUDA tensor (any
-    leading shape; the last dimension is ``cols``)."""
-    cols = x.shape[-1]
-    rows = x.numel() // cols
-    rc = lib().attn_quantize_mxfp8(_ptr(x), _ptr(codes), _ptr(scales), rows, cols,
-                                   _stream_handle(stream, x.device))
+    leading shape; the last dimension is ``cols``, a multiple of 32): codes
+    uint8 [rows, cols], scales uint8 [rows, cols / 32] (E8M0)."""
+    cols = x.shape[-1] if x.dim() > 0 else 0
+    rows, cols = _check_quant_args(x, codes, scales, cols, cols // 32)
+    with torch.cuda.device(x.device):
+        rc = lib().attn_quantize_mxfp8(_ptr(x), _ptr(codes), _ptr(scales), rows, cols,
+                                       _stream_handle(stream, x.device))
     if rc != 0:
         raise AttnError(rc, "attn_quantize_mxfp8")
 
@@ -280,10 +304,11 @@ def attn_quantize_nvfp4(x, codes, scales, stream=None):
     shape; cols a multiple of 16): codes uint8 [rows, cols / 2] (two E2M1
     codes per byte, low nibble first), scales uint8 [rows, cols / 16]
     (unsigned E4M3)."""
-    cols = x.shape[-1]
-    rows = x.numel() // cols
-    rc = lib().attn_quantize_nvfp4(_ptr(x), _ptr(codes), _ptr(scales), rows, cols,
-                                   _stream_handle(stream, x.device))
+    cols = x.shape[-1] if x.dim() > 0 else 0
+    rows, cols = _check_quant_args(x, codes, scales, cols // 2, cols // 16)
+    with torch.cuda.device(x.device):
+        rc = lib().attn_quantize_nvfp4(_ptr(x), _ptr(codes), _ptr(scales), rows, cols,
+                                       _stream_handle(stream, x.device))
     if rc != 0:
         raise AttnError(rc, "attn_quantize_nvfp4")
 
@@ -293,10 +318,11 @@ def attn_quantize_mxfp8_rotated(x, signs, codes, scales, stream=None):
     CUDA tensor (cols 64 or 128; any leading shape): signs fp32 [cols] (+-1)
     on the device; codes uint8 [rows, cols], scales uint8 [rows, cols / 32]
     (``attn_quantize_mxfp8_rotated``)."""
-    cols = x.shape[-1]
-    rows = x.numel() // cols
-    rc = lib().attn_quantize_mxfp8_rotated(_ptr(x), _ptr(signs), _ptr(codes), _ptr(scales), rows,
-                                           cols, _stream_handle(stream, x.device))
+    cols = x.shape[-1] if x.dim() > 0 else 0
+    rows, cols = _check_quant_args(x, codes, scales, cols, cols // 32, signs=signs)
+    with torch.cuda.device(x.device):
+        rc = lib().attn_quantize_mxfp8_rotated(_ptr(x), _ptr(signs), _ptr(codes), _ptr(scales),
+                                               rows, cols, _stream_handle(stream, x.device))
     if rc != 0:
         raise AttnError(rc, "attn_quantize_mxfp8_rotated")
 
@@ -319,9 +345,12 @@ def attn_timing_read() -> tuple[float, float]:
 
 
 def attn_get_device_error(workspace, stream=None) -> int:
+    if not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
     v = ctypes.c_int32(0)
-    rc = lib().attn_get_device_error(_ptr(workspace), _stream_handle(stream, workspace.device),
-                                     ctypes.byref(v))
+    with torch.cuda.device(workspace.device):
+        rc = lib().attn_get_device_error(_ptr(workspace),
+                                         _stream_handle(stream, workspace.device), ctypes.byref(v))
     if rc != 0:
         raise AttnError(rc, "attn_get_device_error")
     return int(v.value)
